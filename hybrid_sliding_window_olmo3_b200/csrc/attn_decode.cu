@@ -1,0 +1,382 @@
+// Split-KV decode attention over the per-layer-type cache, plus the combine.
+//
+// "Olmo 3 7B" (inference-research record), serviceability join: a local layer's
+// decode reads exactly `window` cache entries (about 1 flop per byte, constant in
+// context) while a full layer's reads grow with the context; one kernel serves
+// both.  "Olmo-3 End-to-End Implementation", "Inference Pipeline": one new token
+// per step attends over the cache.  GQA ("Case Study: OLMo 3", ingredient 1):
+// query head h reads key/value head h / (H/G), so one CTA serves the R = H/G
+// query heads of a key/value head and reads each cache row once for all of them.
+//
+// HBM-bound design: grid = (kv head g, split, sequence b) with g fastest, so
+// neighbouring CTAs stream neighbouring rows of the [slots, G, d] cache.  A
+// producer warp feeds 32-key tiles of K and V through a 4-stage TMA/mbarrier
+// ring; 4 compute warps run the dot products with 16-byte shared loads, reduce
+// them with warp shuffles (d/8 lanes per key) and keep an online softmax per lane
+// group in fp32.  Each CTA writes one (max, sum, unnormalised output) partial
+// per query head; the combine kernel merges the partials with log-sum-exp
+// weights.
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace olmo3 {
+
+constexpr int kDecStages = 4;
+constexpr int kDecWarps = 4;  // compute warps; one more warp produces
+constexpr int kDecThreads = (kDecWarps + 1) * 32;
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <int D, int R>
+struct DecodeSmem {
+  static constexpr int kTileBytes = kDecodeTile * D * 2;          // one K (or V) tile
+  static constexpr int kPipeBytes = kDecStages * 2 * kTileBytes;  // K and V rings
+  static constexpr int kGroups = kDecWarps * (32 / (D / 8));      // lane groups per CTA
+  static constexpr int kMergeBytes = kGroups * R * (D + 2) * 4;
+  static constexpr int kBytes = kPipeBytes > kMergeBytes ? kPipeBytes : kMergeBytes;
+};
+
+__device__ __forceinline__ int valid_keys(int L, int layer_type, int window) {
+  return layer_type == OLMO3_SLIDING ? min(L, window) : L;
+}
+
+template <int D, int R>
+__global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(
+    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+    const __nv_bfloat16 *__restrict__ q, const int64_t *__restrict__ seq_base, const int32_t *__restrict__ kv_len,
+    int capacity, int layer_type, int window, int H, int chunk, int n_splits, float scale_log2,
+    float *__restrict__ ws_o, float *__restrict__ ws_ml, int *err) {
+  using S = DecodeSmem<D, R>;
+  constexpr int LPK = D / 8;                        // lanes per key (8 features each)
+  constexpr int KPW = 32 / LPK;                     // keys per warp pass
+  constexpr int KEYS_PER_WARP = kDecodeTile / kDecWarps;
+  constexpr int NIT = KEYS_PER_WARP / KPW;
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ uint64_t full_bar[kDecStages], empty_bar[kDecStages];
+  __shared__ int s_abort;
+
+  const int g = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
+  const int L = kv_len[b];
+  const int n = valid_keys(L, layer_type, window);
+  if (L < 1 || n > capacity || n > n_splits * chunk) {
+    if (split == 0 && g == 0 && threadIdx.x == 0) set_dev_error(err, OLMO3_DEVERR_KV_LEN);
+    return;  // the combine writes zeros for this sequence
+  }
+  const int k_begin = split * chunk;
+  if (k_begin >= n) return;
+  const int k_end = min(n, k_begin + chunk);
+  const int ntiles = (k_end - k_begin + kDecodeTile - 1) / kDecodeTile;
+  const int64_t base = seq_base[b];
+
+  __nv_bfloat16 *sK = reinterpret_cast<__nv_bfloat16 *>(smem);
+  __nv_bfloat16 *sV = sK + kDecStages * kDecodeTile * D;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kDecStages; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], kDecWarps);
+    }
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  const int lg = lane / LPK;  // lane group (key) inside the warp
+  const int li = lane % LPK;  // features li*8 .. li*8+7
+  float m[R], l[R], o[R][8];
+  bool ok = true;
+
+  if (warp == kDecWarps) {
+    // ---------------- producer: one elected lane issues TMA ----------------
+    if (lane == 0) {
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      int issued = 0;
+      for (int i = 0; i < ntiles; ++i) {
+        const int st = i % kDecStages;
+        if (i >= kDecStages && !mbar_wait(&empty_bar[st], ((i / kDecStages) & 1) ^ 1, &s_abort)) {
+          ok = false;
+          break;
+        }
+        const int row = static_cast<int>(base + k_begin + i * kDecodeTile);
+        mbar_arrive_expect_tx(&full_bar[st], 2 * S::kTileBytes);
+        tma_load_3d(sK + st * kDecodeTile * D, &tmK, &full_bar[st], 0, g, row);
+        tma_load_3d(sV + st * kDecodeTile * D, &tmV, &full_bar[st], 0, g, row);
+        ++issued;
+      }
+      if (!ok) {
+        s_abort = 1;
+        set_dev_error(err, OLMO3_DEVERR_TIMEOUT);
+        // let the copies still in flight land before the CTA's shared memory goes away
+        for (int j = max(0, issued - kDecStages); j < issued; ++j)
+          mbar_wait(&full_bar[j % kDecStages], (j / kDecStages) & 1, nullptr);
+      }
+    }
+  } else {
+    // ---------------- compute warps ----------------
+    float qf[R][8];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const uint4 u = *reinterpret_cast<const uint4 *>(q + (static_cast<int64_t>(b) * H + g * R + r) * D + li * 8);
+      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = bf2_to_f2(w4[j]);
+        qf[r][2 * j] = f.x * scale_log2;
+        qf[r][2 * j + 1] = f.y * scale_log2;
+      }
+      m[r] = -INFINITY;
+      l[r] = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) o[r][j] = 0.f;
+    }
+
+    for (int i = 0; i < ntiles; ++i) {
+      const int st = i % kDecStages;
+      if (!__all_sync(0xffffffffu, mbar_wait(&full_bar[st], (i / kDecStages) & 1, &s_abort))) {
+        ok = false;
+        break;
+      }
+      const __nv_bfloat16 *kt = sK + st * kDecodeTile * D;
+      const __nv_bfloat16 *vt = sV + st * kDecodeTile * D;
+      const int key_base = k_begin + i * kDecodeTile;
+
+      float s[R][NIT];
+#pragma unroll
+      for (int it = 0; it < NIT; ++it) {
+        const int kk = warp * KEYS_PER_WARP + it * KPW + lg;
+        const uint4 u = *reinterpret_cast<const uint4 *>(kt + kk * D + li * 8);
+        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+        float kf[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = bf2_to_f2(w4[j]);
+          kf[2 * j] = f.x;
+          kf[2 * j + 1] = f.y;
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          float a = 0.f;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) a = fmaf(qf[r][j], kf[j], a);
+          s[r][it] = a;
+        }
+      }
+#pragma unroll
+      for (int off = LPK / 2; off > 0; off >>= 1) {
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+          for (int it = 0; it < NIT; ++it) s[r][it] += __shfl_xor_sync(0xffffffffu, s[r][it], off);
+      }
+      float p[R][NIT];
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        float mt = -INFINITY;
+#pragma unroll
+        for (int it = 0; it < NIT; ++it) {
+          const int key = key_base + warp * KEYS_PER_WARP + it * KPW + lg;
+          if (key >= k_end) s[r][it] = -INFINITY;
+          mt = fmaxf(mt, s[r][it]);
+        }
+        const float mn = fmaxf(m[r], mt);
+        if (mn == -INFINITY) {  // nothing valid seen yet by this lane group
+#pragma unroll
+          for (int it = 0; it < NIT; ++it) p[r][it] = 0.f;
+          continue;
+        }
+        const float alpha = fast_exp2(m[r] - mn);
+        float rs = 0.f;
+#pragma unroll
+        for (int it = 0; it < NIT; ++it) {
+          p[r][it] = fast_exp2(s[r][it] - mn);
+          rs += p[r][it];
+        }
+        l[r] = l[r] * alpha + rs;
+        m[r] = mn;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) o[r][j] *= alpha;
+      }
+#pragma unroll
+      for (int it = 0; it < NIT; ++it) {
+        const int kk = warp * KEYS_PER_WARP + it * KPW + lg;
+        const uint4 u = *reinterpret_cast<const uint4 *>(vt + kk * D + li * 8);
+        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+        float vf[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = bf2_to_f2(w4[j]);
+          vf[2 * j] = f.x;
+          vf[2 * j + 1] = f.y;
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) o[r][j] = fmaf(p[r][it], vf[j], o[r][j]);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[st]);
+    }
+    if (!ok && lane == 0) {
+      s_abort = 1;
+      set_dev_error(err, OLMO3_DEVERR_TIMEOUT);
+    }
+  }
+  __syncthreads();  // every tile consumed (or drained): the rings can be reused
+  if (s_abort) return;
+
+  // ---------------- merge the lane groups' partials ----------------
+  float *sm_m = reinterpret_cast<float *>(smem);
+  float *sm_l = sm_m + S::kGroups * R;
+  float *sm_o = sm_l + S::kGroups * R;
+  if (warp < kDecWarps) {
+    const int grp = warp * KPW + lg;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (li == 0) {
+        sm_m[grp * R + r] = m[r];
+        sm_l[grp * R + r] = l[r];
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) sm_o[(grp * R + r) * D + li * 8 + j] = o[r][j];
+    }
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < R * D; idx += kDecThreads) {
+    const int r = idx / D, dim = idx % D;
+    float M = -INFINITY;
+    for (int gi = 0; gi < S::kGroups; ++gi) M = fmaxf(M, sm_m[gi * R + r]);
+    float acc = 0.f, den = 0.f;
+    for (int gi = 0; gi < S::kGroups; ++gi) {
+      const float mg = sm_m[gi * R + r];
+      const float w = (mg == -INFINITY) ? 0.f : fast_exp2(mg - M);
+      acc += w * sm_o[(gi * R + r) * D + dim];
+      den += w * sm_l[gi * R + r];
+    }
+    const int64_t slot = (static_cast<int64_t>(b) * H + g * R + r) * n_splits + split;
+    ws_o[slot * D + dim] = acc;
+    if (dim == 0) {
+      ws_ml[slot * 2] = M;
+      ws_ml[slot * 2 + 1] = den;
+    }
+  }
+}
+
+// Merges the split partials of one (sequence, query head): out = sum_s w_s o_s /
+// sum_s w_s l_s with w_s = 2^(m_s - max m).  Writes zeros for a sequence whose
+// kv_len was rejected.
+template <int D>
+__global__ void __launch_bounds__(D) attn_decode_combine_kernel(const int32_t *__restrict__ kv_len, int capacity,
+                                                                 int layer_type, int window, int H, int chunk,
+                                                                 int n_splits, const float *__restrict__ ws_o,
+                                                                 const float *__restrict__ ws_ml,
+                                                                 __nv_bfloat16 *__restrict__ out,
+                                                                 float *__restrict__ lse_out) {
+  const int h = blockIdx.x, b = blockIdx.y, dim = threadIdx.x;
+  const int L = kv_len[b];
+  const int n = valid_keys(L, layer_type, window);
+  const int64_t bh = static_cast<int64_t>(b) * H + h;
+  if (L < 1 || n > capacity || n > n_splits * chunk) {
+    out[bh * D + dim] = __float2bfloat16_rn(0.f);
+    if (lse_out != nullptr && dim == 0) lse_out[bh] = -INFINITY;
+    return;
+  }
+  const int ns = (n + chunk - 1) / chunk;
+  const float *ml = ws_ml + bh * n_splits * 2;
+  const float *po = ws_o + bh * n_splits * D;
+  float M = -INFINITY;
+  for (int s = 0; s < ns; ++s) M = fmaxf(M, ml[2 * s]);
+  float acc = 0.f, den = 0.f;
+  for (int s = 0; s < ns; ++s) {
+    const float w = fast_exp2(ml[2 * s] - M);
+    acc += w * po[static_cast<int64_t>(s) * D + dim];
+    den += w * ml[2 * s + 1];
+  }
+  out[bh * D + dim] = __float2bfloat16_rn(den > 0.f ? acc / den : 0.f);
+  if (lse_out != nullptr && dim == 0) lse_out[bh] = (M + log2f(den)) * 0.69314718055994531f;
+}
+
+DecodePlan plan_decode(int B, int G, int n_max, int num_splits) {
+  DecodePlan pl;
+  const int64_t tiles = (static_cast<int64_t>(n_max) + kDecodeTile - 1) / kDecodeTile;
+  int64_t splits;
+  if (num_splits > 0) {
+    splits = num_splits;
+  } else {
+    // aim at >= 8 waves of 3 CTAs per SM on 148 SMs, with at least 4 tiles per CTA
+    const int64_t target = 148 * 3 * 8;
+    const int64_t pairs = static_cast<int64_t>(B) * G;
+    splits = (target + pairs - 1) / pairs;
+    const int64_t max_splits = (tiles + 3) / 4;
+    if (splits > max_splits) splits = max_splits;
+  }
+  if (splits < 1) splits = 1;
+  if (splits > tiles) splits = tiles;
+  const int64_t tiles_per_split = (tiles + splits - 1) / splits;
+  pl.chunk = static_cast<int>(tiles_per_split * kDecodeTile);
+  pl.n_splits = static_cast<int>((n_max + static_cast<int64_t>(pl.chunk) - 1) / pl.chunk);
+  return pl;
+}
+
+template <int D, int R>
+static cudaError_t launch_rd(const CUtensorMap &tmK, const CUtensorMap &tmV, const void *q, int H,
+                             const olmo3_kv_cache &c, const int32_t *kv_len, const DecodePlan &pl, void *out,
+                             float *lse_out, float scale, float *ws, int *err, cudaStream_t stream) {
+  using S = DecodeSmem<D, R>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(attn_decode_split_kernel<D, R>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, S::kBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int B = c.B;
+  float *ws_o = ws;
+  float *ws_ml = ws + static_cast<int64_t>(B) * H * pl.n_splits * D;
+  const float scale_log2 = scale * 1.4426950408889634f;
+  dim3 grid(c.G, pl.n_splits, B);
+  attn_decode_split_kernel<D, R><<<grid, kDecThreads, S::kBytes, stream>>>(
+      tmK, tmV, static_cast<const __nv_bfloat16 *>(q), c.seq_base, kv_len, c.capacity, c.layer_type, c.window, H,
+      pl.chunk, pl.n_splits, scale_log2, ws_o, ws_ml, err);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  attn_decode_combine_kernel<D><<<dim3(H, B), D, 0, stream>>>(kv_len, c.capacity, c.layer_type, c.window, H,
+                                                              pl.chunk, pl.n_splits, ws_o, ws_ml,
+                                                              static_cast<__nv_bfloat16 *>(out), lse_out);
+  return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_d(int R, const CUtensorMap &tmK, const CUtensorMap &tmV, const void *q, int H,
+                            const olmo3_kv_cache &c, const int32_t *kv_len, const DecodePlan &pl, void *out,
+                            float *lse_out, float scale, float *ws, int *err, cudaStream_t stream) {
+  switch (R) {
+    case 1: return launch_rd<D, 1>(tmK, tmV, q, H, c, kv_len, pl, out, lse_out, scale, ws, err, stream);
+    case 2: return launch_rd<D, 2>(tmK, tmV, q, H, c, kv_len, pl, out, lse_out, scale, ws, err, stream);
+    case 3: return launch_rd<D, 3>(tmK, tmV, q, H, c, kv_len, pl, out, lse_out, scale, ws, err, stream);
+    case 4: return launch_rd<D, 4>(tmK, tmV, q, H, c, kv_len, pl, out, lse_out, scale, ws, err, stream);
+    case 5: return launch_rd<D, 5>(tmK, tmV, q, H, c, kv_len, pl, out, lse_out, scale, ws, err, stream);
+    case 6: return launch_rd<D, 6>(tmK, tmV, q, H, c, kv_len, pl, out, lse_out, scale, ws, err, stream);
+    case 7: return launch_rd<D, 7>(tmK, tmV, q, H, c, kv_len, pl, out, lse_out, scale, ws, err, stream);
+    case 8: return launch_rd<D, 8>(tmK, tmV, q, H, c, kv_len, pl, out, lse_out, scale, ws, err, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_attn_decode(const CUtensorMap &tmK, const CUtensorMap &tmV, const void *q, int H,
+                               const olmo3_kv_cache &c, const int32_t *kv_len, const DecodePlan &plan, void *out,
+                               float *lse_out, float scale, float *ws, int *err, cudaStream_t stream) {
+  const int R = H / c.G;
+  if (c.d == 64) return launch_d<64>(R, tmK, tmV, q, H, c, kv_len, plan, out, lse_out, scale, ws, err, stream);
+  return launch_d<128>(R, tmK, tmV, q, H, c, kv_len, plan, out, lse_out, scale, ws, err, stream);
+}
+
+}  // namespace olmo3

@@ -1,0 +1,46 @@
+// Host-side launchers of the kernels, called by the C ABI in olmo3_abi.cu after
+// argument validation.  Each returns a cudaError_t from the launch.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "olmo3.h"
+
+namespace olmo3 {
+
+struct RopeTable {
+  double inv_freq[64];  // theta^(-2i/d), i < d/2
+};
+
+cudaError_t launch_qknorm_rope(const void *q, const void *k, const void *v, int in_dtype, const float *gain_q,
+                               const float *gain_k, void *q_out, void *k_out, void *v_out,
+                               const int32_t *pos_offset, int B, int T, int H, int G, int d, float eps,
+                               const RopeTable &tab, cudaStream_t stream);
+
+cudaError_t launch_kv_append(const olmo3_kv_cache &c, const void *k_new, const void *v_new,
+                             const int32_t *pos_offset, int T, int32_t *slot_out, int *err, cudaStream_t stream);
+
+cudaError_t launch_attn_mask(int T, int window, int layer_type, uint8_t *out, cudaStream_t stream);
+
+// Split plan of the decode kernel (keys per split and splits per (sequence, head)).
+struct DecodePlan {
+  int chunk;
+  int n_splits;
+};
+DecodePlan plan_decode(int B, int G, int n_max, int num_splits);
+constexpr int kDecodeTile = 32;  // keys per pipeline stage
+
+cudaError_t launch_attn_decode(const CUtensorMap &tmK, const CUtensorMap &tmV, const void *q, int H,
+                               const olmo3_kv_cache &c, const int32_t *kv_len, const DecodePlan &plan, void *out,
+                               float *lse_out, float scale, float *ws, int *err, cudaStream_t stream);
+
+constexpr int kPrefillBM = 128;  // query rows per CTA
+constexpr int kPrefillBN = 128;  // keys per tile
+
+cudaError_t launch_attn_prefill(const CUtensorMap &tmQ, const CUtensorMap &tmK, const CUtensorMap &tmV, void *out,
+                                float *lse_out, int B, int T, int H, int G, int d, int layer_type, int window,
+                                float scale, int *err, cudaStream_t stream);
+
+}  // namespace olmo3

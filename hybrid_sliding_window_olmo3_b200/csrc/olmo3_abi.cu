@@ -1,0 +1,181 @@
+// The C ABI of libolmo3 (declared in include/olmo3.h): host-side argument
+// validation, TMA tensor-map encoding and kernel launches.  Nothing here
+// allocates device memory; every buffer belongs to the caller.
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "internal.h"
+#include "olmo3.h"
+
+using namespace olmo3;
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool encoder_ready() {
+  std::call_once(g_encode_once, [] {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode != nullptr;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool valid_d(int d) { return d == 64 || d == 128; }
+bool valid_type(int t) { return t == OLMO3_SLIDING || t == OLMO3_FULL; }
+cudaStream_t as_stream(void *s) { return static_cast<cudaStream_t>(s); }
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? OLMO3_OK : OLMO3_ERR_CUDA; }
+
+// bf16 tensor of rank `rank` (dims innermost first, byte strides of dims 1..rank-1).
+bool encode_bf16(CUtensorMap *tm, const void *base, int rank, const cuuint64_t *dims, const cuuint64_t *strides,
+                 const cuuint32_t *box, CUtensorMapSwizzle swz) {
+  if (!encoder_ready()) return false;
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int validate_cache(const olmo3_kv_cache *c) {
+  if (c == nullptr || c->k == nullptr || c->v == nullptr || c->seq_base == nullptr) return OLMO3_ERR_INVALID_ARG;
+  if (!valid_type(c->layer_type) || c->B < 0 || c->G < 1 || c->capacity < 1 || c->total_slots < 1 ||
+      c->window < 1)
+    return OLMO3_ERR_INVALID_ARG;
+  if (!valid_d(c->d)) return OLMO3_ERR_UNSUPPORTED;
+  if (c->layer_type == OLMO3_SLIDING && c->capacity != c->window) return OLMO3_ERR_INVALID_ARG;
+  if (c->total_slots >= (int64_t(1) << 31)) return OLMO3_ERR_UNSUPPORTED;
+  if (!aligned16(c->k) || !aligned16(c->v)) return OLMO3_ERR_INVALID_ARG;
+  return OLMO3_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *olmo3_status_string(int status) {
+  switch (status) {
+    case OLMO3_OK: return "ok";
+    case OLMO3_ERR_INVALID_ARG: return "invalid argument";
+    case OLMO3_ERR_UNSUPPORTED: return "unsupported shape";
+    case OLMO3_ERR_WORKSPACE: return "workspace missing or too small";
+    case OLMO3_ERR_CUDA: return "CUDA error";
+    default: return "unknown status";
+  }
+}
+
+int olmo3_layer_types(int n_layers, uint8_t *out_host) {
+  if (n_layers < 0 || (n_layers > 0 && out_host == nullptr)) return OLMO3_ERR_INVALID_ARG;
+  for (int l = 0; l < n_layers; ++l)
+    out_host[l] = (l % 4 == 3 || l == n_layers - 1) ? OLMO3_FULL : OLMO3_SLIDING;
+  return OLMO3_OK;
+}
+
+int olmo3_attn_mask(int T, int window, int layer_type, uint8_t *out_dev, void *stream) {
+  if (T < 0 || !valid_type(layer_type) || (layer_type == OLMO3_SLIDING && window < 1)) return OLMO3_ERR_INVALID_ARG;
+  if (T == 0) return OLMO3_OK;
+  if (out_dev == nullptr) return OLMO3_ERR_INVALID_ARG;
+  return cuda_status(launch_attn_mask(T, window, layer_type, out_dev, as_stream(stream)));
+}
+
+int olmo3_qknorm_rope(const void *q, const void *k, const void *v, int in_dtype, const float *gain_q,
+                      const float *gain_k, void *q_out, void *k_out, void *v_out, const int32_t *pos_offset, int B,
+                      int T, int H, int G, int d, float eps, double theta, void *stream) {
+  if (B < 0 || T < 0 || H < 1 || G < 1 || !(eps >= 0.f) || !(theta > 0.0) ||
+      (in_dtype != OLMO3_F32 && in_dtype != OLMO3_BF16))
+    return OLMO3_ERR_INVALID_ARG;
+  if (!valid_d(d)) return OLMO3_ERR_UNSUPPORTED;
+  if (H * d > 8192 || G * d > 8192) return OLMO3_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(B) * T == 0) return OLMO3_OK;
+  if (static_cast<int64_t>(B) * T > 0x7fffffffLL) return OLMO3_ERR_UNSUPPORTED;
+  if (!q || !k || !gain_q || !gain_k || !q_out || !k_out || !pos_offset || (v_out && !v))
+    return OLMO3_ERR_INVALID_ARG;
+  const void *ptrs[] = {q, k, gain_q, gain_k, q_out, k_out};
+  for (const void *p : ptrs)
+    if (!aligned16(p)) return OLMO3_ERR_INVALID_ARG;
+  if (v_out && (!aligned16(v) || !aligned16(v_out))) return OLMO3_ERR_INVALID_ARG;
+  RopeTable tab;
+  for (int i = 0; i < 64; ++i) tab.inv_freq[i] = i < d / 2 ? pow(theta, -2.0 * i / d) : 0.0;
+  return cuda_status(launch_qknorm_rope(q, k, v, in_dtype, gain_q, gain_k, q_out, k_out, v_out, pos_offset, B, T,
+                                        H, G, d, eps, tab, as_stream(stream)));
+}
+
+int olmo3_kv_append(const olmo3_kv_cache *c, const void *k_new, const void *v_new, const int32_t *pos_offset,
+                    int T, int32_t *slot_out, int *err_dev, void *stream) {
+  int st = validate_cache(c);
+  if (st != OLMO3_OK) return st;
+  if (T < 0 || c->B > 65535) return OLMO3_ERR_INVALID_ARG;
+  if (T == 0 || c->B == 0) return OLMO3_OK;
+  if (!k_new || !v_new || !pos_offset || !aligned16(k_new) || !aligned16(v_new)) return OLMO3_ERR_INVALID_ARG;
+  return cuda_status(launch_kv_append(*c, k_new, v_new, pos_offset, T, slot_out, err_dev, as_stream(stream)));
+}
+
+int olmo3_attn_prefill(const void *q, const void *k, const void *v, void *out, int B, int T, int H, int G, int d,
+                       int layer_type, int window, float scale, float *lse_out, int *err_dev, void *stream) {
+  if (B < 0 || T < 0 || H < 1 || G < 1 || !valid_type(layer_type) || window < 1 || !isfinite(scale))
+    return OLMO3_ERR_INVALID_ARG;
+  if (!valid_d(d) || H % G != 0) return OLMO3_ERR_UNSUPPORTED;
+  if (B > 65535 || (T + kPrefillBM - 1) / kPrefillBM > 65535) return OLMO3_ERR_UNSUPPORTED;
+  if (B == 0 || T == 0) return OLMO3_OK;
+  if (!q || !k || !v || !out) return OLMO3_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return OLMO3_ERR_INVALID_ARG;
+  CUtensorMap tmQ, tmK, tmV;
+  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kPrefillBM), 1};
+  const cuuint64_t dq[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+  const cuuint64_t sq[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)T * H * d * 2};
+  const cuuint64_t dk[4] = {(cuuint64_t)d, (cuuint64_t)G, (cuuint64_t)T, (cuuint64_t)B};
+  const cuuint64_t sk[3] = {(cuuint64_t)d * 2, (cuuint64_t)G * d * 2, (cuuint64_t)T * G * d * 2};
+  if (!encode_bf16(&tmQ, q, 4, dq, sq, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_bf16(&tmK, k, 4, dk, sk, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_bf16(&tmV, v, 4, dk, sk, box, CU_TENSOR_MAP_SWIZZLE_128B))
+    return OLMO3_ERR_CUDA;
+  return cuda_status(launch_attn_prefill(tmQ, tmK, tmV, out, lse_out, B, T, H, G, d, layer_type, window, scale,
+                                         err_dev, as_stream(stream)));
+}
+
+size_t olmo3_attn_decode_workspace_size(int B, int H, int G, int d, int max_kv_len, int layer_type, int window,
+                                        int num_splits) {
+  if (B < 0 || H < 1 || G < 1 || !valid_d(d) || H % G != 0 || max_kv_len < 1 || !valid_type(layer_type) ||
+      window < 1 || num_splits < 0)
+    return 0;
+  const int n_max = layer_type == OLMO3_SLIDING ? (max_kv_len < window ? max_kv_len : window) : max_kv_len;
+  const DecodePlan pl = plan_decode(B, G, n_max, num_splits);
+  return static_cast<size_t>(B) * H * pl.n_splits * (d + 2) * sizeof(float);
+}
+
+int olmo3_attn_decode(const void *q, int H, const olmo3_kv_cache *c, const int32_t *kv_len, int max_kv_len,
+                      void *out, float *lse_out, float scale, int num_splits, void *workspace, size_t ws_bytes,
+                      int *err_dev, void *stream) {
+  int st = validate_cache(c);
+  if (st != OLMO3_OK) return st;
+  if (H < 1 || max_kv_len < 1 || num_splits < 0 || !isfinite(scale)) return OLMO3_ERR_INVALID_ARG;
+  if (H % c->G != 0 || H / c->G > 8) return OLMO3_ERR_UNSUPPORTED;
+  if (c->B > 65535) return OLMO3_ERR_UNSUPPORTED;
+  if (c->B == 0) return OLMO3_OK;
+  if (!q || !kv_len || !out || !aligned16(q) || !aligned16(out)) return OLMO3_ERR_INVALID_ARG;
+  const size_t need =
+      olmo3_attn_decode_workspace_size(c->B, H, c->G, c->d, max_kv_len, c->layer_type, c->window, num_splits);
+  if (workspace == nullptr || ws_bytes < need || !aligned16(workspace)) return OLMO3_ERR_WORKSPACE;
+  const int n_max = c->layer_type == OLMO3_SLIDING ? (max_kv_len < c->window ? max_kv_len : c->window) : max_kv_len;
+  const DecodePlan pl = plan_decode(c->B, c->G, n_max, num_splits);
+  if (pl.n_splits > 65535) return OLMO3_ERR_UNSUPPORTED;
+  CUtensorMap tmK, tmV;
+  const cuuint64_t dims[3] = {(cuuint64_t)c->d, (cuuint64_t)c->G, (cuuint64_t)c->total_slots};
+  const cuuint64_t strides[2] = {(cuuint64_t)c->d * 2, (cuuint64_t)c->G * c->d * 2};
+  const cuuint32_t box[3] = {(cuuint32_t)c->d, 1, (cuuint32_t)kDecodeTile};
+  if (!encode_bf16(&tmK, c->k, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_bf16(&tmV, c->v, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return OLMO3_ERR_CUDA;
+  return cuda_status(launch_attn_decode(tmK, tmV, q, H, *c, kv_len, pl, out, lse_out, scale,
+                                        static_cast<float *>(workspace), err_dev, as_stream(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,392 @@
+"""GPU parity: every kernel of libolmo3, called through the C ABI, against the
+fp64 oracle on the same seeded inputs.
+
+Bars: masks, layer types, cache slots and cache contents bit-exact; QK-norm +
+RoPE within bf16 rounding (|err| <= 2^-8 |ref| + 1e-4); attention outputs
+max-abs <= 2e-2 and mean-abs <= 2e-3; LSE within 5e-3.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.olmo3_oracle as O
+from conftest import read_golden
+from hybrid_sliding_window_olmo3_b200 import olmo3 as L
+from hybrid_sliding_window_olmo3_b200 import workloads as WL
+
+pytestmark = pytest.mark.gpu
+
+TYP = {L.SLIDING: O.SLIDING, L.FULL: O.FULL}
+MAX_ABS, MEAN_ABS, LSE_ABS = 2e-2, 2e-3, 5e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    L.lib()
+    yield
+    torch.cuda.synchronize()
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def bf16(a: np.ndarray, dev="cuda") -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dev).to(torch.bfloat16)
+
+
+def close_attn(got, ref, what=""):
+    err = np.abs(np.asarray(got, np.float64) - np.asarray(ref, np.float64))
+    assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, f"{what}: max {err.max():.3e} mean {err.mean():.3e}"
+
+
+def close_qk(got, ref, what=""):
+    err = np.abs(got - ref)
+    bound = 2.0 ** -8 * np.abs(ref) + 1e-4
+    bad = err > bound
+    assert not bad.any(), f"{what}: {bad.sum()} elements beyond bf16 rounding, worst {err.max():.3e}"
+
+
+def new_err():
+    return torch.zeros(1, dtype=torch.int32, device="cuda")
+
+
+# ---------------------------------------------------------------------------
+# masks
+# ---------------------------------------------------------------------------
+def test_mask_table_T5_window2_bit_exact():
+    want = np.array([[int(x) for x in r] for r in read_golden("mask_T5_window2.txt")], dtype=np.uint8)
+    got = L.attn_mask(5, 2, L.SLIDING).cpu().numpy()
+    np.testing.assert_array_equal(got, want)
+
+
+@pytest.mark.parametrize("T,W,typ", [(1, 1, L.SLIDING), (37, 5, L.SLIDING), (300, 128, L.SLIDING),
+                                     (300, 128, L.FULL), (1000, 4096, L.SLIDING), (513, 1, L.SLIDING)])
+def test_mask_bit_exact_vs_oracle(T, W, typ):
+    got = L.attn_mask(T, W, typ).cpu().numpy().astype(bool)
+    want = O.causal_mask(T) if typ == L.FULL else O.sliding_window_mask(T, W)
+    np.testing.assert_array_equal(got, want)
+
+
+# ---------------------------------------------------------------------------
+# K1: QK-norm + RoPE
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("B,T,H,G,d,dt,offs", [
+    (1, 24, 2, 1, 64, "f32", [0]),
+    (2, 5, 32, 32, 128, "bf16", [0, 65530]),
+    (2, 3, 40, 8, 128, "bf16", [7, 131072]),
+    (1, 130, 4, 2, 128, "bf16", [1000]),
+    (3, 2, 2, 2, 64, "f32", [0, 4095, 4096]),
+])
+def test_qknorm_rope_parity(B, T, H, G, d, dt, offs):
+    rng = np.random.default_rng(100 + B * T + H)
+    q = rng.standard_normal((B, T, H, d)) * 3
+    k = rng.standard_normal((B, T, G, d)) * 3
+    v = rng.standard_normal((B, T, G, d))
+    gq, gk = rng.uniform(0.5, 1.5, H * d), rng.uniform(0.5, 1.5, G * d)
+    if dt == "bf16":
+        tq, tk, tv = bf16(q), bf16(k), bf16(v)
+    else:
+        tq, tk, tv = (torch.from_numpy(x.astype(np.float32)).cuda() for x in (q, k, v))
+    q, k, v = f64(tq), f64(tk), f64(tv)   # exact values the GPU sees
+    tgq = torch.from_numpy(gq.astype(np.float32)).cuda()
+    tgk = torch.from_numpy(gk.astype(np.float32)).cuda()
+    gq, gk = f64(tgq), f64(tgk)
+    pos = torch.tensor(offs, dtype=torch.int32, device="cuda")
+    qh, kh, vo = L.qknorm_rope(tq, tk, tgq, tgk, pos, 1e-6, 5e5, v=tv)
+    positions = np.array(offs)[:, None] + np.arange(T)[None, :]
+    rq, rk = O.qk_norm_rope(q, k, gq, gk, positions, 1e-6, 5e5)
+    close_qk(f64(qh), rq, "q_hat")
+    close_qk(f64(kh), rk, "k_hat")
+    # v is only cast to bf16 (round to nearest even), bit for bit
+    assert torch.equal(vo.cpu(), tv.cpu().to(torch.bfloat16))
+
+
+def test_qknorm_rope_in_place():
+    rng = np.random.default_rng(7)
+    B, T, H, G, d = 2, 9, 8, 4, 128
+    tq, tk = bf16(rng.standard_normal((B, T, H, d))), bf16(rng.standard_normal((B, T, G, d)))
+    q0, k0 = f64(tq), f64(tk)
+    gq = torch.rand(H * d, device="cuda") + 0.5
+    gk = torch.rand(G * d, device="cuda") + 0.5
+    pos = torch.tensor([3, 40000], dtype=torch.int32, device="cuda")
+    L.qknorm_rope(tq, tk, gq, gk, pos, q_out=tq, k_out=tk)
+    rq, rk = O.qk_norm_rope(q0, k0, f64(gq), f64(gk), np.array([3, 40000])[:, None] + np.arange(T))
+    close_qk(f64(tq), rq, "in-place q")
+    close_qk(f64(tk), rk, "in-place k")
+
+
+# ---------------------------------------------------------------------------
+# K2: KV append (bit-exact slots and contents; canary rows around the cache)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("typ,W,cap,B,T,offs", [
+    (L.SLIDING, 4, 4, 1, 16, [0]),
+    (L.SLIDING, 4, 4, 2, 1, [16, 3]),
+    (L.SLIDING, 64, 64, 3, 50, [0, 30, 100]),
+    (L.SLIDING, 64, 64, 2, 200, [5, 0]),
+    (L.FULL, 4096, 200, 2, 17, [0, 150]),
+    (L.FULL, 4096, 64, 1, 64, [0]),
+])
+def test_kv_append_bit_exact(typ, W, cap, B, T, offs):
+    G, d, pad = 2, 128, 3
+    rng = np.random.default_rng(200 + T)
+    kn, vn = bf16(rng.standard_normal((B, T, G, d))), bf16(rng.standard_normal((B, T, G, d)))
+    total = B * cap + 2 * pad
+    sentinel = 1234.0
+    ck = torch.full((total, G, d), sentinel, dtype=torch.bfloat16, device="cuda")
+    cv = torch.full((total, G, d), -sentinel, dtype=torch.bfloat16, device="cuda")
+    base = torch.tensor([pad + b * cap for b in range(B)], dtype=torch.int64, device="cuda")
+    cache = L.KVCache(typ, B, G, d, W, capacity=cap, k=ck, v=cv, seq_base=base)
+    slot_out = torch.empty((B, T), dtype=torch.int32, device="cuda")
+    err = new_err()
+    L.kv_append(cache, kn, vn, torch.tensor(offs, dtype=torch.int32, device="cuda"), slot_out, err)
+    want_slots = O.append_slots(offs, T, TYP[typ], cap)
+    np.testing.assert_array_equal(slot_out.cpu().numpy(), want_slots)
+    assert err.item() == 0
+    # expected cache: the oracle's replay of every row in order
+    exp_k = np.full((total, G, d), sentinel)
+    exp_v = np.full((total, G, d), -sentinel)
+    kn64, vn64 = f64(kn), f64(vn)
+    for b in range(B):
+        oc = O.KVCache(TYP[typ], cap, G, d)
+        oc.append(range(offs[b], offs[b] + T), kn64[b], vn64[b])
+        for s in range(cap):
+            if oc.pos[s] >= 0:
+                exp_k[pad + b * cap + s] = oc.k[s]
+                exp_v[pad + b * cap + s] = oc.v[s]
+    np.testing.assert_array_equal(f64(ck), exp_k)
+    np.testing.assert_array_equal(f64(cv), exp_v)
+
+
+def test_kv_append_capacity_error_skips_rows():
+    B, T, G, d, cap = 1, 6, 1, 64, 8
+    kn = bf16(np.ones((B, T, G, d)))
+    ck = torch.zeros((cap, G, d), dtype=torch.bfloat16, device="cuda")
+    cv = torch.zeros_like(ck)
+    cache = L.KVCache(L.FULL, B, G, d, 4096, capacity=cap, k=ck, v=cv)
+    slot_out = torch.empty((B, T), dtype=torch.int32, device="cuda")
+    err = new_err()
+    L.kv_append(cache, kn, kn, torch.tensor([5], dtype=torch.int32, device="cuda"), slot_out, err)
+    assert slot_out.cpu().tolist() == [[5, 6, 7, -1, -1, -1]]
+    assert err.item() & L.DEVERR_CAPACITY
+    assert f64(ck)[5:].min() == 1.0 and f64(ck)[:5].max() == 0.0
+
+
+# ---------------------------------------------------------------------------
+# K3: prefill attention (tcgen05)
+# ---------------------------------------------------------------------------
+PREFILL_CASES = [
+    # B, T, H, G, d, type, window, q scale
+    (1, 16, 2, 1, 64, L.SLIDING, 4, 1.0),
+    (1, 16, 2, 1, 64, L.FULL, 4, 1.0),
+    (1, 300, 4, 2, 128, L.SLIDING, 200, 1.0),
+    (2, 257, 5, 1, 128, L.SLIDING, 128, 1.0),
+    (1, 384, 2, 2, 64, L.FULL, 4096, 1.0),
+    (1, 255, 2, 2, 128, L.SLIDING, 256, 1.0),
+    (1, 256, 2, 2, 128, L.SLIDING, 256, 1.0),
+    (1, 257, 2, 2, 128, L.SLIDING, 256, 1.0),
+    (1, 1, 1, 1, 128, L.SLIDING, 4096, 1.0),
+    (1, 700, 2, 1, 128, L.SLIDING, 1, 1.0),
+    (1, 640, 10, 2, 128, L.SLIDING, 129, 1.0),
+    (3, 1000, 2, 2, 128, L.FULL, 4096, 1.0),
+    (1, 777, 4, 4, 128, L.SLIDING, 300, 4.0),   # peaky logits: exercises the O rescale
+    (1, 520, 2, 1, 64, L.FULL, 4096, 6.0),
+]
+
+
+@pytest.mark.parametrize("B,T,H,G,d,typ,W,qs", PREFILL_CASES)
+def test_prefill_parity(B, T, H, G, d, typ, W, qs):
+    rng = np.random.default_rng(300 + T + H + d)
+    tq = bf16(rng.standard_normal((B, T, H, d)) * qs)
+    tk = bf16(rng.standard_normal((B, T, G, d)))
+    tv = bf16(rng.standard_normal((B, T, G, d)))
+    lse = torch.empty((B, H, T), dtype=torch.float32, device="cuda")
+    err = new_err()
+    out = L.attn_prefill(tq, tk, tv, typ, W, lse=lse, err=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    ro, rl = O.prefill_attention(f64(tq), f64(tk), f64(tv), TYP[typ], W)
+    close_attn(f64(out), ro, "prefill out")
+    assert np.abs(lse.cpu().numpy() - rl).max() <= LSE_ABS
+
+
+def _sampled_prefill(B, T, H, G, d, seed, rows):
+    for typ in (L.SLIDING, L.FULL):
+        q, k, v, _, _ = WL.qkv_bf16(B, T, H, G, d, seed, layer=typ)
+        tq, tk, tv = q.cuda(), k.cuda(), v.cuda()
+        out = L.attn_prefill(tq, tk, tv, typ, 4096)
+        torch.cuda.synchronize()
+        got = f64(out[:, rows])
+        ro, _ = O.prefill_attention(f64(q), f64(k), f64(v), TYP[typ], 4096, rows=rows)
+        close_attn(got, ro, f"sampled prefill type {typ}")
+
+
+def test_prefill_7b_full_size_sampled_rows():
+    rng = np.random.default_rng(1)
+    rows = sorted(set([0, 1, 127, 128, 129, 4094, 4095, 4096, 4097, 6000, 8190, 8191] +
+                      rng.integers(0, 8192, 8).tolist()))
+    _sampled_prefill(1, 8192, 32, 32, 128, WL.WORKLOADS["7b-prefill"].seed, rows)
+
+
+def test_prefill_32b_full_size_sampled_rows():
+    rng = np.random.default_rng(2)
+    rows = sorted(set([0, 255, 4095, 4096, 8191] + rng.integers(0, 8192, 5).tolist()))
+    _sampled_prefill(2, 8192, 40, 8, 128, WL.WORKLOADS["32b-prefill"].seed, rows)
+
+
+# ---------------------------------------------------------------------------
+# K4: decode attention over ring / linear caches
+# ---------------------------------------------------------------------------
+def _decode_case(B, H, G, d, typ, W, lens, seed, num_splits=0, q_scale=1.0):
+    rng = np.random.default_rng(seed)
+    cap = W if typ == L.SLIDING else max(lens) + 5
+    ocs, base = [], []
+    ck = torch.zeros((B * cap, G, d), dtype=torch.bfloat16, device="cuda")
+    cv = torch.zeros_like(ck)
+    for b, n in enumerate(lens):
+        oc = O.KVCache(TYP[typ], cap, G, d)
+        first = max(0, n - cap) if typ == L.SLIDING else 0   # earlier rows are overwritten anyway
+        rows_k = f64(bf16(rng.standard_normal((n - first, G, d)), "cpu"))
+        rows_v = f64(bf16(rng.standard_normal((n - first, G, d)), "cpu"))
+        oc.append(range(first, n), rows_k, rows_v)
+        valid = oc.valid()
+        ck[b * cap:(b + 1) * cap][torch.from_numpy(valid).cuda()] = bf16(oc.k[valid])
+        cv[b * cap:(b + 1) * cap][torch.from_numpy(valid).cuda()] = bf16(oc.v[valid])
+        ocs.append(oc)
+    cache = L.KVCache(typ, B, G, d, W, capacity=cap, k=ck, v=cv)
+    tq = bf16(rng.standard_normal((B, H, d)) * q_scale)
+    kv_len = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    lse = torch.empty((B, H), dtype=torch.float32, device="cuda")
+    err = new_err()
+    out = L.attn_decode(tq, cache, kv_len, max(lens), lse=lse, err=err, num_splits=num_splits)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    ro, rl = O.decode_attention(f64(tq), ocs, [n - 1 for n in lens], TYP[typ], W)
+    close_attn(f64(out), ro, "decode out")
+    assert np.abs(lse.cpu().numpy() - rl).max() <= LSE_ABS
+
+
+@pytest.mark.parametrize("typ", [L.SLIDING, L.FULL])
+@pytest.mark.parametrize("B,H,G,d,W,lens", [
+    (6, 2, 1, 64, 4, [1, 3, 4, 5, 8, 9]),
+    (5, 4, 2, 128, 256, [255, 256, 257, 512, 513]),
+    (3, 10, 2, 128, 4096, [1000, 33, 4097]),
+    (2, 8, 1, 128, 64, [100, 64]),
+    (4, 6, 2, 64, 128, [1, 2, 127, 300]),
+])
+def test_decode_parity(typ, B, H, G, d, W, lens):
+    _decode_case(B, H, G, d, typ, W, lens, seed=400 + sum(lens))
+
+
+@pytest.mark.parametrize("splits", [1, 3, 7, 200])
+def test_decode_split_count_does_not_change_the_result(splits):
+    _decode_case(3, 4, 4, 128, L.FULL, 4096, [5000, 1, 777], seed=9, num_splits=splits, q_scale=3.0)
+
+
+def test_decode_bad_kv_len_sets_error_and_zeroes_only_that_sequence():
+    B, H, G, d, cap = 3, 2, 2, 128, 64
+    ck = bf16(np.random.default_rng(3).standard_normal((B * cap, G, d)))
+    cache = L.KVCache(L.FULL, B, G, d, 4096, capacity=cap, k=ck, v=ck.clone())
+    q = bf16(np.random.default_rng(4).standard_normal((B, H, d)))
+    err = new_err()
+    out = L.attn_decode(q, cache, torch.tensor([10, 0, 65], dtype=torch.int32, device="cuda"), 65, err=err)
+    torch.cuda.synchronize()
+    assert err.item() & L.DEVERR_KV_LEN
+    o = f64(out)
+    assert np.all(o[1] == 0) and np.all(o[2] == 0) and np.abs(o[0]).sum() > 0
+
+
+def _sampled_decode(B, H, G, d, lens, seed, check):
+    """Random caches on the device; the oracle recomputes the sequences in `check`."""
+    for typ in (L.SLIDING, L.FULL):
+        cap = 4096 if typ == L.SLIDING else int(max(lens))
+        n_slots = B * cap
+        ck = WL.randn_bf16((n_slots, G, d), seed * 10 + typ, "cuda")
+        cv = WL.randn_bf16((n_slots, G, d), seed * 10 + typ + 5, "cuda")
+        cache = L.KVCache(typ, B, G, d, 4096, capacity=cap, k=ck, v=cv)
+        q = WL.randn_bf16((B, H, d), seed + 77, "cuda")
+        kv_len = torch.tensor(lens, dtype=torch.int32, device="cuda")
+        err = new_err()
+        out = L.attn_decode(q, cache, kv_len, int(max(lens)), err=err)
+        torch.cuda.synchronize()
+        assert err.item() == 0
+        for b in check:
+            n = int(lens[b])
+            oc = O.KVCache(TYP[typ], cap, G, d)
+            first = max(0, n - cap) if typ == L.SLIDING else 0
+            slots = [(p % cap if typ == L.SLIDING else p) for p in range(first, n)]
+            rows_k = f64(ck[b * cap:(b + 1) * cap])[slots]
+            rows_v = f64(cv[b * cap:(b + 1) * cap])[slots]
+            oc.append(range(first, n), rows_k, rows_v)
+            ro, _ = O.decode_attention(f64(q[b:b + 1]), [oc], [n - 1], TYP[typ], 4096)
+            close_attn(f64(out[b:b + 1]), ro, f"decode seq {b} type {typ}")
+        del ck, cv, cache
+        torch.cuda.empty_cache()
+
+
+def test_decode_7b_full_size_sampled():
+    wl = WL.WORKLOADS["7b-decode"]
+    _sampled_decode(32, 32, 32, 128, [wl.context + 1] * 32, wl.seed, check=[0, 31])
+
+
+def test_decode_32b_full_size_sampled():
+    wl = WL.WORKLOADS["32b-decode"]
+    _sampled_decode(8, 40, 8, 128, [wl.context + 1] * 8, wl.seed, check=[0, 7])
+
+
+def test_decode_ragged_7b_full_size_sampled():
+    wl = WL.WORKLOADS["ragged-7b-decode"]
+    lens = WL.ragged_lengths(64, wl.seed).tolist()
+    order = np.argsort(lens)
+    _sampled_decode(64, 32, 32, 128, lens, wl.seed, check=[int(order[0]), int(order[-1]), 5])
+
+
+# ---------------------------------------------------------------------------
+# The toy configuration end to end: 6 layers, prefill 16 tokens, 8 decode steps
+# ---------------------------------------------------------------------------
+def test_toy_pipeline_full_parity():
+    wl = WL.WORKLOADS["toy"]
+    sh = wl.shape
+    T0, steps = wl.T, wl.steps
+    layers = WL.toy_layer_inputs(wl.seed, T0 + steps)
+    types = L.layer_types(sh.n_layers)
+    assert [TYP[t] for t in types] == O.layer_types(sh.n_layers)
+    for li, typ in enumerate(types):
+        x = layers[li]
+        q, k, v = (torch.from_numpy(x[n]).cuda() for n in ("q", "k", "v"))
+        gq, gk = torch.from_numpy(x["gain_q"]).cuda(), torch.from_numpy(x["gain_k"]).cuda()
+        # oracle over all 24 tokens
+        pos_all = np.arange(T0 + steps)[None, :]
+        rq, rk = O.qk_norm_rope(x["q"], x["k"], x["gain_q"], x["gain_k"], pos_all, sh.eps, sh.theta)
+        rv = x["v"].astype(np.float64)
+        # GPU prefill
+        zero = torch.zeros(1, dtype=torch.int32, device="cuda")
+        qh, kh, vb = L.qknorm_rope(q[:, :T0].contiguous(), k[:, :T0].contiguous(), gq, gk, zero, sh.eps,
+                                   sh.theta, v=v[:, :T0].contiguous())
+        close_qk(f64(qh), rq[:, :T0], "toy q_hat")
+        close_qk(f64(kh), rk[:, :T0], "toy k_hat")
+        cache = L.KVCache(typ, 1, sh.G, sh.d, sh.window, capacity=T0 + steps)
+        L.kv_append(cache, kh, vb, zero)
+        out = L.attn_prefill(qh, kh, vb, typ, sh.window)
+        ro, _ = O.prefill_attention(rq[:, :T0], rk[:, :T0], rv[:, :T0], TYP[typ], sh.window)
+        close_attn(f64(out), ro, f"toy prefill layer {li}")
+        # oracle cache
+        oc = O.KVCache(TYP[typ], cache.capacity, sh.G, sh.d)
+        oc.append(range(T0), rk[0, :T0], rv[0, :T0])
+        for s in range(steps):
+            p = T0 + s
+            pos = torch.tensor([p], dtype=torch.int32, device="cuda")
+            qh1, kh1, vb1 = L.qknorm_rope(q[:, p:p + 1].contiguous(), k[:, p:p + 1].contiguous(), gq, gk, pos,
+                                          sh.eps, sh.theta, v=v[:, p:p + 1].contiguous())
+            L.kv_append(cache, kh1, vb1, pos)
+            o1 = L.attn_decode(qh1[:, 0].contiguous(), cache, torch.tensor([p + 1], dtype=torch.int32,
+                                                                          device="cuda"), p + 1)
+            oc.append([p], rk[0, p:p + 1], rv[0, p:p + 1])
+            ro1, _ = O.decode_attention(rq[:, p], [oc], [p], TYP[typ], sh.window)
+            close_attn(f64(o1), ro1, f"toy decode layer {li} step {s}")
+            full = O.full_recompute_last_row(rq[:, :p + 1], rk[:, :p + 1], rv[:, :p + 1], TYP[typ], sh.window)
+            close_attn(f64(o1), full, f"toy decode vs recompute layer {li} step {s}")
