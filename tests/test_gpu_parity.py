@@ -136,7 +136,7 @@ def test_kv_append_bit_exact(typ, W, cap, B, T, offs):
     rng = np.random.default_rng(200 + T)
     kn, vn = bf16(rng.standard_normal((B, T, G, d))), bf16(rng.standard_normal((B, T, G, d)))
     total = B * cap + 2 * pad
-    sentinel = 1234.0
+    sentinel = 4096.0  # exactly representable in bf16
     ck = torch.full((total, G, d), sentinel, dtype=torch.bfloat16, device="cuda")
     cv = torch.full((total, G, d), -sentinel, dtype=torch.bfloat16, device="cuda")
     base = torch.tensor([pad + b * cap for b in range(B)], dtype=torch.int64, device="cuda")
