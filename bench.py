@@ -44,7 +44,7 @@ CSRC = os.path.join(ROOT, "hybrid_sliding_window_olmo3_b200", "csrc")
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="7b-prefill",
@@ -52,6 +52,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--batch", type=int, default=0, help="override B of a decode workload (small profiling captures)")
     return ap.parse_args()
 
 
@@ -282,14 +283,14 @@ class PrefillStep:
 class DecodeStep:
     """One decode token per sequence through every layer of the model pattern."""
 
-    def __init__(self, name, dev, stream):
+    def __init__(self, name, dev, stream, batch=0):
         from hybrid_sliding_window_olmo3_b200 import olmo3 as L
         from hybrid_sliding_window_olmo3_b200 import workloads as WL
         self.L = L
         wl = WL.WORKLOADS[name]
         sh = wl.shape
         self.wl, self.sh, self.dev, self.stream = wl, sh, dev, stream
-        B, H, G, d, W = wl.B, sh.H, sh.G, sh.d, sh.window
+        B, H, G, d, W = (batch or wl.B), sh.H, sh.G, sh.d, sh.window
         self.B = B
         if wl.ragged:
             lens = WL.ragged_lengths(B, wl.seed)
@@ -434,8 +435,8 @@ class DecodeStep:
                           f"one sliding and one full layer), {el:.1f} s of oracle time; numpy, single thread"}
 
 
-def make_workload(name, dev, stream):
-    return PrefillStep(name, dev, stream) if name.endswith("prefill") else DecodeStep(name, dev, stream)
+def make_workload(name, dev, stream, batch=0):
+    return PrefillStep(name, dev, stream) if name.endswith("prefill") else DecodeStep(name, dev, stream, batch)
 
 
 # --------------------------------------------------------------------------
@@ -450,7 +451,7 @@ def run_ours(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
     stream = torch.cuda.current_stream(dev)
-    wk = make_workload(args.workload, dev, stream)
+    wk = make_workload(args.workload, dev, stream, args.batch)
     peaks, peak_src = load_peaks()
 
     def barrier():
@@ -459,12 +460,12 @@ def run_ours(args):
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    for _ in range(args.warmup):
-        wk.step()
-    barrier()
     work = 0.0
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
+    with ClockSampler(local) as clk:  # started before the warm-up so that it is sampling when timing begins
+        for _ in range(args.warmup):
+            wk.step()
+        barrier()
         e0.record(stream)
         for _ in range(args.steps):
             work += wk.work_per_step()
@@ -537,7 +538,7 @@ def run_reference(args):
     if dev is None:
         print(json.dumps({"impl": "reference", "unavailable": "the sampled workload is generated on a CUDA device"}))
         return
-    wk = make_workload(args.workload, dev, torch.cuda.current_stream(dev))
+    wk = make_workload(args.workload, dev, torch.cuda.current_stream(dev), args.batch)
     per = []
     for i in range(args.warmup + args.steps):
         cb = wk.cpu_baseline(max(2.0, min(8.0, 150.0 / (args.warmup + args.steps))))

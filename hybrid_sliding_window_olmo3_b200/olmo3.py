@@ -250,3 +250,33 @@ def attn_decode(q: torch.Tensor, cache: KVCache, kv_len: torch.Tensor, max_kv_le
         _p(q), H, ctypes.byref(s), _p(kv_len), max_kv_len, _p(out), _p(lse), sc, num_splits,
         _p(workspace), workspace.numel() * workspace.element_size(), _p(err), _stream(stream)))
     return out
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def attn_decode_noalloc(q: torch.Tensor, cache: KVCache, kv_len: torch.Tensor, max_kv_len: int,
+                        scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                        lse: Optional[torch.Tensor] = None, num_splits: int = 0,
+                        err: Optional[torch.Tensor] = None, stream=None):
+    """attn_decode without a workspace: the library's own fixed scratch buffer
+    (NOALLOC_SCRATCH_BYTES per GPU) holds the split partials.  For callers that
+    cannot allocate; concurrent calls on different streams race on the buffer."""
+    fn = lib().olmo3_attn_decode_noalloc
+    fn.argtypes = [_vp, _i, ctypes.POINTER(CacheStruct), _vp, _i, _vp, _vp, ctypes.c_float, _i, _vp, _vp]
+    fn.restype = _i
+    B, H, d = q.shape
+    _dev(q, "q", torch.bfloat16, (cache.B, H, cache.d))
+    _dev(kv_len, "kv_len", torch.int32, (cache.B,))
+    if out is None:
+        out = torch.empty_like(q)
+    _dev(out, "out", torch.bfloat16, (B, H, d))
+    if lse is not None:
+        _dev(lse, "lse", torch.float32, (B, H))
+    if err is not None:
+        _dev(err, "err", torch.int32)
+    sc = 1.0 / math.sqrt(d) if scale is None else scale
+    s = cache.struct()
+    _check("olmo3_attn_decode_noalloc", fn(_p(q), H, ctypes.byref(s), _p(kv_len), max_kv_len, _p(out), _p(lse), sc,
+                                           num_splits, _p(err), _stream(stream)))
+    return out

@@ -203,6 +203,34 @@ int olmo3_attn_decode(const void *q, int H, const olmo3_kv_cache *c,
                       float scale, int num_splits, void *workspace, size_t ws_bytes,
                       int *err_dev, void *stream);
 
+/*
+ * olmo3_attn_decode_noalloc - olmo3_attn_decode for callers that cannot allocate
+ * device memory.  The pages have no counterpart: this is a library convenience.
+ *   Some callers only ever receive input and output buffers from a host framework
+ *   (a plugin or custom-operator interface with no workspace argument), or run
+ *   without an allocator of their own, where a cudaMalloc would synchronise the
+ *   device or break a fixed memory budget.  This entry point takes the same
+ *   arguments as olmo3_attn_decode minus the workspace, and keeps the split-KV
+ *   partials in a buffer of OLMO3_NOALLOC_SCRATCH_BYTES that the library holds as
+ *   a file-scope device array (present on every GPU that loads the library, until
+ *   the process exits).  It calls no cudaMalloc, cudaFree or allocating routine.
+ *   Limit: a call whose olmo3_attn_decode_workspace_size() exceeds
+ *   OLMO3_NOALLOC_SCRATCH_BYTES returns OLMO3_ERR_WORKSPACE and launches nothing
+ *   (a smaller num_splits lowers the need).
+ *   Set-up: the first call on each device looks up the buffer's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call before
+ *   any stream capture.
+ *   Sharing: every call uses the same buffer and it keeps the last call's
+ *   contents (harmless: each value read is written earlier in the same call).
+ *   Calls that overlap on the GPU (other streams, other threads) race on it:
+ *   order them on one stream or serialise them.
+ */
+#define OLMO3_NOALLOC_SCRATCH_BYTES (16u << 20)
+int olmo3_attn_decode_noalloc(const void *q, int H, const olmo3_kv_cache *c,
+                              const int32_t *kv_len, int max_kv_len, void *out,
+                              float *lse_out, float scale, int num_splits, int *err_dev,
+                              void *stream);
+
 /* olmo3_status_string - a static English description of a status code. */
 const char *olmo3_status_string(int status);
 
