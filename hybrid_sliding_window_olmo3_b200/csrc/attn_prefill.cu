@@ -5,24 +5,28 @@
 // OLMo 3", "The architecture", ingredient 4: three layers in four are sliding;
 // ingredient 1: grouped-query attention (head h reads key/value head h/(H/G)).
 //
-// One CTA computes a 128-row query tile of one head.  Only the key tiles that
-// intersect the band [t - window + 1, t] of its rows are visited, so a sliding
-// layer costs O(T * window) instead of O(T^2); only the two edge tiles of the
-// band apply the mask predicate.
+// One CTA computes 256 query rows (two 128-row tiles, A and B) of one head.  Only
+// the key tiles that intersect the band [t - window + 1, t] of its rows are
+// visited, so a sliding layer costs O(T * window) instead of O(T^2); only the
+// edge tiles of each band apply the mask predicate.
 //
-// Warp roles (192 threads):
-//   warps 0-3  softmax + epilogue: thread i owns query row i = TMEM lane i.
-//   warp  4    TMA producer: Q once, then K and V tiles into a 2-stage ring.
-//   warp  5    TMEM allocator and MMA issuer (one thread).
-// Tensor memory (512 columns): S double buffer at columns [0,128) and [128,256)
-// (fp32 128x128 score tiles), O accumulator at [256, 256 + d).
-// Per key tile j: S_j = Q K_j^T on the tensor core while the softmax warps turn
-// S_{j-1} into P_{j-1} (bf16, written to shared memory in the 128-byte-swizzled
-// K-major layout the MMA reads); then O += P_j V_j with V read MN-major.  The
-// running max is only raised (and O rescaled in TMEM) when a row's max grows by
-// more than 2^8, so P stays <= 256 and most tiles skip the rescale.
+// Warp roles (384 threads, three warpgroups):
+//   WG0 (warps 0-3)  softmax + epilogue of tile A: thread i owns row i = TMEM lane i.
+//   WG1 (warps 4-7)  the same for tile B.
+//   WG2 warp 8       TMA producer: both Q tiles once, then K_j, V_j, K_j+1, ... into
+//                    a 3-slot ring (each slot holds one 128-key K or V tile).
+//       warp 9       TMEM allocator and MMA issuer (one thread).
+// WG2 gives registers to the softmax warpgroups (setmaxnreg).
+// Tensor memory (512 columns): S_A [0,128), S_B [128,256) fp32 score tiles,
+// O_A [256, 256+d), O_B [256+d, 256+2d) fp32 accumulators.
+// Tensor-core order per key tile j:  PV_A(j), S_A(j+1), PV_B(j), S_B(j+1): while
+// one softmax warpgroup turns its S into P (bf16, 128-byte-swizzled K-major in
+// shared memory) the tensor core works for the other tile, so the two
+// warpgroups alternate against a busy tensor core.  A row's running max is only
+// raised (and O rescaled in TMEM) when it grows by more than 2^8, so P <= 256 and
+// most tiles skip the rescale.
 // Every wait is bounded: on a timeout the CTA records OLMO3_DEVERR_TIMEOUT,
-// drains its copies in flight, frees its tensor memory and exits.
+// drains its copies and MMAs in flight, frees its tensor memory and exits.
 #include <math.h>
 
 #include "common.cuh"
@@ -30,12 +34,14 @@
 
 namespace olmo3 {
 
-constexpr int kBM = kPrefillBM;
-constexpr int kBN = kPrefillBN;
-constexpr int kPfStages = 2;
-constexpr int kPfThreads = 192;
+constexpr int kBM = kPrefillBM;  // rows per query tile
+constexpr int kBN = kPrefillBN;  // keys per key tile
+constexpr int kRing = 3;
+constexpr int kPfThreads = 384;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
+constexpr uint32_t kSoftmaxRegs = 224;  // 2 x 128 x 224 + 128 x 56 = 384 x 168 (the launch budget)
+constexpr uint32_t kControlRegs = 56;
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -43,76 +49,105 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 template <int D>
 struct PfLayout {
-  static constexpr int kQBytes = kBM * D * 2;  // D/64 swizzled blocks of 128 rows x 128 B
-  static constexpr int kKBytes = kBN * D * 2;
-  static constexpr int kVBytes = kBN * D * 2;
-  static constexpr int kPBytes = kBM * kBN * 2;  // 2 swizzled blocks of 128 rows x 128 B
+  static constexpr int kQBytes = kBM * D * 2;   // one query tile: D/64 swizzled blocks of 128 rows x 128 B
+  static constexpr int kKVBytes = kBN * D * 2;  // one K or V tile
+  static constexpr int kPBytes = kBM * kBN * 2;  // one P tile: 2 swizzled blocks of 128 rows x 128 B
   static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kOffQ + kQBytes;
-  static constexpr int kOffV = kOffK + kPfStages * kKBytes;
-  static constexpr int kOffP = kOffV + kPfStages * kVBytes;
-  static constexpr int kUsed = kOffP + kPBytes;
-  // at least 120 KB so that one CTA (and one 512-column TMEM allocation) fits an SM
-  static constexpr int kDynBytes = (kUsed + 1024) > 120 * 1024 ? (kUsed + 1024) : 120 * 1024;
+  static constexpr int kOffRing = kOffQ + 2 * kQBytes;
+  static constexpr int kOffP = kOffRing + kRing * kKVBytes;
+  static constexpr int kUsed = kOffP + 2 * kPBytes;
+  static constexpr int kDynBytes = kUsed + 1024;  // + alignment slack for the 1024-byte swizzle atoms
 };
+
+// Tiles (in units of kBN keys) a query tile [r0, r1] needs: [first, last].
+__device__ __forceinline__ void band_tiles(int r0, int r1, bool is_full, int window, int &first, int &last) {
+  const int64_t lo = static_cast<int64_t>(r0) - window + 1;
+  first = (is_full || lo < 0) ? 0 : static_cast<int>(lo / kBN);
+  last = r1 / kBN;
+}
 
 template <int D>
 __global__ void __launch_bounds__(kPfThreads, 1)
     attn_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, __nv_bfloat16 *__restrict__ out,
                         float *__restrict__ lse_out, int T, int H, int G, int layer_type, int window,
-                        float scale_log2, int n_qtiles, int *err) {
+                        float scale_log2, int n_blocks, int *err) {
   using LY = PfLayout<D>;
   constexpr int NDB = D / 64;  // 64-feature (128-byte) blocks per row
   constexpr uint32_t IDESC_S = idesc_bf16_f32(kBM, kBN, 0);
   constexpr uint32_t IDESC_O = idesc_bf16_f32(kBM, D, 1);
 
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t q_full, k_full[kPfStages], v_full[kPfStages], kv_empty[kPfStages];
-  __shared__ uint64_t s_full[2], s_free[2], p_full, o_done, mma_drain;
+  __shared__ uint64_t q_full, ring_full[kRing], ring_empty[kRing];
+  __shared__ uint64_t s_full[2], p_full[2], o_done[2], mma_drain;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
 
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sQ = smem + LY::kOffQ;
-  uint8_t *sK = smem + LY::kOffK;
-  uint8_t *sV = smem + LY::kOffV;
+  uint8_t *sRing = smem + LY::kOffRing;
   uint8_t *sP = smem + LY::kOffP;
 
   const int h = blockIdx.x;
-  const int qt = n_qtiles - 1 - static_cast<int>(blockIdx.y);  // longest rows first
+  const int qb = n_blocks - 1 - static_cast<int>(blockIdx.y);  // longest rows first
   const int b = blockIdx.z;
   const int g = h / (H / G);
-  const int q0 = qt * kBM;
-  const int q_last = min(q0 + kBM, T) - 1;
+  const int q0 = qb * 2 * kBM;
   const bool is_full = layer_type == OLMO3_FULL;
-  const int64_t lo_key = static_cast<int64_t>(q0) - window + 1;
-  const int64_t first_key = (is_full || lo_key < 0) ? 0 : lo_key;
-  const int kt_first = static_cast<int>(first_key / kBN);
-  const int n_kt = q_last / kBN - kt_first + 1;
+
+  // key-tile ranges: the union [kt_lo, kt_lo + n_kt) and, per query tile w, [lo_w, hi_w] inside it
+  int lo[2], hi[2];
+#pragma unroll
+  for (int w = 0; w < 2; ++w) {
+    const int r0 = q0 + w * kBM;
+    if (r0 < T) {
+      int f, l;
+      band_tiles(r0, min(r0 + kBM, T) - 1, is_full, window, f, l);
+      lo[w] = f;
+      hi[w] = l;
+    } else {
+      lo[w] = 1;
+      hi[w] = 0;  // empty: every row of this tile is past the sequence
+    }
+  }
+  const int kt_lo = lo[0];
+  const int kt_hi = hi[1] >= lo[1] ? hi[1] : hi[0];
+  const int n_kt = kt_hi - kt_lo + 1;
+#pragma unroll
+  for (int w = 0; w < 2; ++w) {
+    lo[w] -= kt_lo;
+    hi[w] -= kt_lo;
+  }
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
   if (threadIdx.x == 0) {
     mbar_init(&q_full, 1);
-    for (int i = 0; i < kPfStages; ++i) {
-      mbar_init(&k_full[i], 1);
-      mbar_init(&v_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(&ring_full[i], 1);
+      mbar_init(&ring_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], kBM);
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&s_full[w], 1);
+      mbar_init(&p_full[w], kBM);
+      mbar_init(&o_done[w], 1);
     }
-    mbar_init(&p_full, kBM);
-    mbar_init(&o_done, 1);
     mbar_init(&mma_drain, 1);
     s_abort = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(&s_tmem, kTmemCols);
     tmem_relinquish();
   }
@@ -121,153 +156,180 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   tc_fence_after();
   const uint32_t tmem = s_tmem;
 
-  if (warp == 4) {
-    // ------------------------------ TMA producer ------------------------------
-    if (lane == 0) {
+  if (warp >= 8) {
+    regs_dec<kControlRegs>();
+    if (warp == 8 && lane == 0) {
+      // ------------------------------ TMA producer ------------------------------
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      mbar_arrive_expect_tx(&q_full, LY::kQBytes);
+      mbar_arrive_expect_tx(&q_full, 2 * LY::kQBytes);
 #pragma unroll
-      for (int db = 0; db < NDB; ++db) tma_load_4d(sQ + db * kBM * 128, &tmQ, &q_full, db * 64, h, q0, b);
+      for (int w = 0; w < 2; ++w)
+#pragma unroll
+        for (int db = 0; db < NDB; ++db)
+          tma_load_4d(sQ + w * LY::kQBytes + db * kBM * 128, &tmQ, &q_full, db * 64, h, q0 + w * kBM, b);
       int issued = 0;
       bool ok = true;
-      for (int j = 0; j < n_kt; ++j) {
-        const int st = j % kPfStages;
-        if (j >= kPfStages && !mbar_wait(&kv_empty[st], ((j / kPfStages) & 1) ^ 1, &s_abort)) {
+      for (int i = 0; i < 2 * n_kt; ++i) {
+        const int slot = i % kRing;
+        if (i >= kRing && !mbar_wait(&ring_empty[slot], ((i / kRing) & 1) ^ 1, &s_abort)) {
           ok = false;
           break;
         }
-        const int k0 = (kt_first + j) * kBN;
-        mbar_arrive_expect_tx(&k_full[st], LY::kKBytes);
+        const int k0 = (kt_lo + (i >> 1)) * kBN;
+        const CUtensorMap *tm = (i & 1) ? &tmV : &tmK;
+        mbar_arrive_expect_tx(&ring_full[slot], LY::kKVBytes);
 #pragma unroll
         for (int db = 0; db < NDB; ++db)
-          tma_load_4d(sK + st * LY::kKBytes + db * kBN * 128, &tmK, &k_full[st], db * 64, g, k0, b);
-        mbar_arrive_expect_tx(&v_full[st], LY::kVBytes);
-#pragma unroll
-        for (int db = 0; db < NDB; ++db)
-          tma_load_4d(sV + st * LY::kVBytes + db * kBN * 128, &tmV, &v_full[st], db * 64, g, k0, b);
+          tma_load_4d(sRing + slot * LY::kKVBytes + db * kBN * 128, tm, &ring_full[slot], db * 64, g, k0, b);
         ++issued;
       }
       if (!ok) {
         s_abort = 1;
         set_dev_error(err, OLMO3_DEVERR_TIMEOUT);
         mbar_wait(&q_full, 0, nullptr);
-        for (int j = max(0, issued - kPfStages); j < issued; ++j) {
-          mbar_wait(&k_full[j % kPfStages], (j / kPfStages) & 1, nullptr);
-          mbar_wait(&v_full[j % kPfStages], (j / kPfStages) & 1, nullptr);
-        }
+        for (int i = max(0, issued - kRing); i < issued; ++i)
+          mbar_wait(&ring_full[i % kRing], (i / kRing) & 1, nullptr);
       }
-    }
-  } else if (warp == 5) {
-    // ------------------------------ MMA issuer ------------------------------
-    if (lane == 0) {
-      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
-      const uint32_t tO = tmem + 256;
+    } else if (warp == 9 && lane == 0) {
+      // ------------------------------ MMA issuer ------------------------------
+      const uint32_t aQ = smem_u32(sQ), aR = smem_u32(sRing), aP = smem_u32(sP);
+      int cnt_pv[2] = {0, 0};
       bool ok = mbar_wait(&q_full, 0, &s_abort);
-      auto issue_s = [&](int j) -> bool {
-        const int st = j % kPfStages, sb = j & 1;
-        if (!mbar_wait(&k_full[st], (j / kPfStages) & 1, &s_abort)) return false;
-        if (j >= 2 && !mbar_wait(&s_free[sb], ((j >> 1) - 1) & 1, &s_abort)) return false;
-        tc_fence_after();
+      auto item_ready = [&](int i) -> bool {
+        return mbar_wait(&ring_full[i % kRing], (i / kRing) & 1, &s_abort);
+      };
+      auto issue_s = [&](int w, int j) {  // S_w = Q_w K_j^T (K_j is item 2j)
+        const uint32_t kb = aR + ((2 * j) % kRing) * LY::kKVBytes;
+        const uint32_t qw = aQ + w * LY::kQBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t qa = aQ + (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
-          const uint32_t ka = aK + st * LY::kKBytes + (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
-          umma_bf16(tmem + sb * kBN, sw128_desc(qa, 16, 1024), sw128_desc(ka, 16, 1024), IDESC_S, kk > 0);
+          const uint32_t off = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
+          umma_bf16(tmem + w * kBN, sw128_desc(qw + off, 16, 1024), sw128_desc(kb + off, 16, 1024), IDESC_S,
+                    kk > 0);
         }
-        umma_commit(&s_full[sb]);
-        return true;
+        umma_commit(&s_full[w]);
       };
-      auto issue_pv = [&](int j) -> bool {
-        const int st = j % kPfStages;
-        if (!mbar_wait(&p_full, j & 1, &s_abort)) return false;
-        if (!mbar_wait(&v_full[st], (j / kPfStages) & 1, &s_abort)) return false;
+      auto issue_pv = [&](int w, int j) -> bool {  // O_w += P_w V_j (V_j is item 2j+1)
+        if (!mbar_wait(&p_full[w], cnt_pv[w] & 1, &s_abort)) return false;
         tc_fence_after();
+        const uint32_t vb = aR + ((2 * j + 1) % kRing) * LY::kKVBytes;
+        const uint32_t pb = aP + w * LY::kPBytes;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint32_t pa = aP + (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
-          const uint32_t va = aV + st * LY::kVBytes + kk * (16 * 128);
-          umma_bf16(tO, sw128_desc(pa, 16, 1024), sw128_desc(va, kBN * 128, 1024), IDESC_O, (j > 0 || kk > 0));
+          umma_bf16(tmem + 256 + w * D, sw128_desc(pb + (kk >> 2) * (kBM * 128) + (kk & 3) * 32, 16, 1024),
+                    sw128_desc(vb + kk * (16 * 128), kBN * 128, 1024), IDESC_O, (cnt_pv[w] > 0 || kk > 0));
         }
-        umma_commit(&kv_empty[st]);
-        umma_commit(&o_done);
+        umma_commit(&o_done[w]);
+        ++cnt_pv[w];
         return true;
       };
-      if (ok) ok = issue_s(0);
+      auto active = [&](int w, int j) { return lo[w] <= j && j <= hi[w]; };
+
+      if (ok) ok = item_ready(0);
+      if (ok) {
+        tc_fence_after();
+        if (active(0, 0)) issue_s(0, 0);
+        if (active(1, 0)) issue_s(1, 0);
+        umma_commit(&ring_empty[0]);
+      }
       for (int j = 0; ok && j < n_kt; ++j) {
-        if (j + 1 < n_kt) ok = issue_s(j + 1);
-        if (ok) ok = issue_pv(j);
+        if (!(ok = item_ready(2 * j + 1))) break;  // V_j
+        tc_fence_after();
+        if (active(0, j) && !(ok = issue_pv(0, j))) break;
+        const bool more = j + 1 < n_kt;
+        if (more) {
+          if (!(ok = item_ready(2 * j + 2))) break;  // K_{j+1}
+          tc_fence_after();
+          if (active(0, j + 1)) issue_s(0, j + 1);
+        }
+        if (active(1, j) && !(ok = issue_pv(1, j))) break;
+        umma_commit(&ring_empty[(2 * j + 1) % kRing]);  // V_j consumed by both PVs
+        if (more) {
+          if (active(1, j + 1)) issue_s(1, j + 1);
+          umma_commit(&ring_empty[(2 * j + 2) % kRing]);  // K_{j+1} consumed by both S
+        }
       }
       if (!ok) {
         s_abort = 1;
         set_dev_error(err, OLMO3_DEVERR_TIMEOUT);
       }
-      // every MMA this thread issued has completed before tensor memory is freed
-      umma_commit(&mma_drain);
+      umma_commit(&mma_drain);  // every MMA issued has completed before tensor memory is freed
       mbar_wait(&mma_drain, 0, nullptr);
     }
   } else {
+    regs_inc<kSoftmaxRegs>();
     // -------------------------- softmax + epilogue --------------------------
-    const int row = threadIdx.x;  // TMEM lane and query row inside the tile
-    const int t = q0 + row;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const int w = warp >> 2;            // query tile of this warpgroup
+    const int row = threadIdx.x & 127;  // TMEM lane and row inside the tile
+    const int r0 = q0 + w * kBM;
+    const int t = r0 + row;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + w * kBN;
+    const uint32_t tO = tmem + lane_off + 256 + w * D;
+    uint8_t *myP = sP + w * LY::kPBytes;
     float m_used = -INFINITY, lsum = 0.f;
+    int cnt = 0;
     bool ok = true;
-    for (int j = 0; j < n_kt; ++j) {
-      const int sb = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], (j >> 1) & 1, &s_abort))) {
+    for (int j = lo[w]; j <= hi[w]; ++j, ++cnt) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[w], cnt & 1, &s_abort))) {
         ok = false;
         break;
       }
       tc_fence_after();
       uint32_t sr[kBN / 32][32];
 #pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) tmem_ld32(tmem + lane_off + sb * kBN + c * 32, sr[c]);
+      for (int c = 0; c < kBN / 32; ++c) tmem_ld32(tS + c * 32, sr[c]);
       tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&s_free[sb]);
 
-      const int k0 = (kt_first + j) * kBN;
-      const bool need_mask = !(k0 + kBN - 1 <= q0 && (is_full || (q0 + kBM - 1) - k0 < window));
-      float mt = -INFINITY;
+      const int k0 = (kt_lo + j) * kBN;
+      const bool need_mask = !(k0 + kBN - 1 <= r0 && (is_full || (r0 + kBM - 1) - k0 < window));
+      if (need_mask) {
 #pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) {
+        for (int c = 0; c < kBN / 32; ++c)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          float x = __uint_as_float(sr[c][i]) * scale_log2;
-          if (need_mask) {
+          for (int i = 0; i < 32; ++i) {
             const int key = k0 + c * 32 + i;
             const bool allowed = key <= t && (is_full || t - key < window);
-            x = allowed ? x : -INFINITY;
+            if (!allowed) sr[c][i] = __float_as_uint(-INFINITY);
           }
-          sr[c][i] = __float_as_uint(x);
-          mt = fmaxf(mt, x);
-        }
       }
-      const float mn = fmaxf(m_used, mt);
-      const bool resc = mn > m_used + kRescaleLog2;  // false while the row has seen nothing
-      float alpha = 1.f;
-      if (resc) {
-        alpha = ex2(m_used - mn);  // 0 when m_used == -inf
-        m_used = mn;
-      }
-      const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
-      float rs = 0.f;
+      // row max of the raw scores: 8 independent chains, then a tree
+      float mx[8];
 #pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) {
+      for (int k = 0; k < 8; ++k) mx[k] = __uint_as_float(sr[k >> 2][(k & 3) * 8]);
+#pragma unroll
+      for (int c = 0; c < kBN / 32; ++c)
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float p = ex2(__uint_as_float(sr[c][i]) - m_eff);
-          rs += p;
+          const int e = c * 32 + i, k = (e >> 3) & 7;
+          mx[k] = fmaxf(mx[k], __uint_as_float(sr[c][i]));
+        }
+      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * scale_log2;
+      const bool resc = mt > m_used + kRescaleLog2;  // false while the row has seen nothing
+      float alpha = 1.f;
+      if (resc) {
+        alpha = ex2(m_used - mt);  // 0 when m_used == -inf
+        m_used = mt;
+      }
+      const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
+      float sm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < kBN / 32; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int e = c * 32 + i, k = (e >> 3) & 7;
+          const float p = ex2(fmaf(__uint_as_float(sr[c][i]), scale_log2, neg_m));
+          sm[k] += p;
           sr[c][i] = __float_as_uint(p);
         }
-      }
-      lsum = lsum * alpha + rs;
+      lsum = lsum * alpha + (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
 
       // P_j overwrites P_{j-1} and O is rescaled: both wait for PV_{j-1}
-      if (j > 0) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&o_done, (j - 1) & 1, &s_abort))) {
+      if (cnt > 0) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&o_done[w], (cnt - 1) & 1, &s_abort))) {
           ok = false;
           break;
         }
@@ -276,11 +338,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t orr[32];
-            tmem_ld32(tmem + lane_off + 256 + c * 32, orr);
+            tmem_ld32(tO + c * 32, orr);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
-            tmem_st32(tmem + lane_off + 256 + c * 32, orr);
+            tmem_st32(tO + c * 32, orr);
           }
           tmem_wait_st();
         }
@@ -296,27 +358,27 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           u.y = f2_to_bf2(__uint_as_float(sr[e / 32][e % 32 + 2]), __uint_as_float(sr[e / 32][e % 32 + 3]));
           u.z = f2_to_bf2(__uint_as_float(sr[e / 32][e % 32 + 4]), __uint_as_float(sr[e / 32][e % 32 + 5]));
           u.w = f2_to_bf2(__uint_as_float(sr[e / 32][e % 32 + 6]), __uint_as_float(sr[e / 32][e % 32 + 7]));
-          *reinterpret_cast<uint4 *>(sP + kb * (kBM * 128) + row * 128 + ((c ^ (row & 7)) * 16)) = u;
+          *reinterpret_cast<uint4 *>(myP + kb * (kBM * 128) + row * 128 + ((c ^ (row & 7)) * 16)) = u;
         }
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&p_full);
+      mbar_arrive(&p_full[w]);
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_done, (n_kt - 1) & 1, &s_abort));
+    if (ok && cnt > 0) ok = __all_sync(0xffffffffu, mbar_wait(&o_done[w], (cnt - 1) & 1, &s_abort));
     if (!ok) {
       if (lane == 0) {
         s_abort = 1;
         set_dev_error(err, OLMO3_DEVERR_TIMEOUT);
       }
-    } else {
+    } else if (cnt > 0) {
       tc_fence_after();
       const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
       __nv_bfloat16 *orow = out + ((static_cast<int64_t>(b) * T + t) * H + h) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t orr[32];
-        tmem_ld32(tmem + lane_off + 256 + c * 32, orr);
+        tmem_ld32(tO + c * 32, orr);
         tmem_wait_ld();
         if (t < T) {
 #pragma unroll
@@ -339,7 +401,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -357,11 +419,11 @@ static cudaError_t launch_pf(const CUtensorMap &tmQ, const CUtensorMap &tmK, con
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const int n_qtiles = (T + kBM - 1) / kBM;
-  dim3 grid(H, n_qtiles, B);
+  const int n_blocks = (T + 2 * kBM - 1) / (2 * kBM);
+  dim3 grid(H, n_blocks, B);
   attn_prefill_kernel<D><<<grid, kPfThreads, LY::kDynBytes, stream>>>(
       tmQ, tmK, tmV, static_cast<__nv_bfloat16 *>(out), lse_out, T, H, G, layer_type, window,
-      scale * 1.4426950408889634f, n_qtiles, err);
+      scale * 1.4426950408889634f, n_blocks, err);
   return cudaGetLastError();
 }
 
