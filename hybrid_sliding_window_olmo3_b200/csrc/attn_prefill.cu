@@ -14,15 +14,18 @@
 //   WG0 (warps 0-3)  softmax + epilogue of tile A: thread i owns row i = TMEM lane i.
 //   WG1 (warps 4-7)  the same for tile B.
 //   WG2 warp 8       TMA producer: both Q tiles once, then K_j, V_j, K_j+1, ... into
-//                    a 3-slot ring (each slot holds one 128-key K or V tile).
+//                    a 4-slot ring (each slot holds one 128-key K or V tile).
 //       warp 9       TMEM allocator and MMA issuer (one thread).
 // WG2 gives registers to the softmax warpgroups (setmaxnreg).
 // Tensor memory (512 columns): S_A [0,128), S_B [128,256) fp32 score tiles,
-// O_A [256, 256+d), O_B [256+d, 256+2d) fp32 accumulators.
+// O_A [256, 256+d), O_B [256+d, 256+2d) fp32 accumulators.  P (bf16, two per
+// 32-bit column) overwrites the first 64 columns of its S tile once S is read,
+// and the PV product takes its A operand straight from tensor memory, so shared
+// memory only carries Q, K and V (the S and PV products both read two operands
+// at 128 rows x 128 columns, which is what the shared-memory bandwidth allows).
 // Tensor-core order per key tile j:  PV_A(j), S_A(j+1), PV_B(j), S_B(j+1): while
-// one softmax warpgroup turns its S into P (bf16, 128-byte-swizzled K-major in
-// shared memory) the tensor core works for the other tile, so the two
-// warpgroups alternate against a busy tensor core.  A row's running max is only
+// one softmax warpgroup turns its S into P the tensor core works for the other
+// tile, so the two warpgroups alternate against a busy tensor core.  A row's running max is only
 // raised (and O rescaled in TMEM) when it grows by more than 2^8, so P <= 256 and
 // most tiles skip the rescale.
 // Every wait is bounded: on a timeout the CTA records OLMO3_DEVERR_TIMEOUT,
@@ -36,17 +39,43 @@ namespace olmo3 {
 
 constexpr int kBM = kPrefillBM;  // rows per query tile
 constexpr int kBN = kPrefillBN;  // keys per key tile
-constexpr int kRing = 3;
+constexpr int kRing = 4;
 constexpr int kPfThreads = 384;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
-constexpr uint32_t kSoftmaxRegs = 224;  // 2 x 128 x 224 + 128 x 56 = 384 x 168 (the launch budget)
-constexpr uint32_t kControlRegs = 56;
+#ifndef OLMO3_PF_CONTROL_REGS
+#define OLMO3_PF_CONTROL_REGS 64
+#endif
+#ifndef OLMO3_PF_EXP2_POLY_EVERY
+#define OLMO3_PF_EXP2_POLY_EVERY 0
+#endif
+// Register split between the control warpgroup and the two softmax warpgroups:
+// 128 x control + 256 x softmax must not exceed 384 x 168 (the launch budget).
+constexpr uint32_t kControlRegs = OLMO3_PF_CONTROL_REGS;
+constexpr uint32_t kSoftmaxRegs = ((384u * 168u - 128u * kControlRegs) / 256u) & ~7u;
+// Every kPolyEvery-th score of a row takes its exp2 on the FMA pipe (exp2_poly)
+// instead of the transcendental unit, which the rest of the exps saturate.
+constexpr int kPolyEvery = OLMO3_PF_EXP2_POLY_EVERY;
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA and integer pipes.  Cody-Waite style range reduction x = j + f
+// with j = round(x) (adding and removing 1.5 * 2^23 rounds to an integer held in
+// the low mantissa bits) and |f| <= 1/2, then a degree-3 polynomial for 2^f whose
+// coefficients are a Remez (minimax relative error) fit on [-1/2, 1/2], max
+// relative error 7.5e-5 (far below the 2^-8 of the bf16 P it feeds); j is added
+// to the exponent field.  x is clamped to >= -126 so the result stays >= 0
+// (2^-126 stands for the exp of a masked score, i.e. 0 at bf16 precision).
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -126.0f);
+  const float t = x + 12582912.0f;
+  const float f = x - (t - 12582912.0f);
+  const float p = fmaf(fmaf(fmaf(0.0551716685f, f, 0.242611125f), f, 0.693260968f), f, 0.999928057f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 template <uint32_t N>
@@ -62,11 +91,9 @@ template <int D>
 struct PfLayout {
   static constexpr int kQBytes = kBM * D * 2;   // one query tile: D/64 swizzled blocks of 128 rows x 128 B
   static constexpr int kKVBytes = kBN * D * 2;  // one K or V tile
-  static constexpr int kPBytes = kBM * kBN * 2;  // one P tile: 2 swizzled blocks of 128 rows x 128 B
   static constexpr int kOffQ = 0;
   static constexpr int kOffRing = kOffQ + 2 * kQBytes;
-  static constexpr int kOffP = kOffRing + kRing * kKVBytes;
-  static constexpr int kUsed = kOffP + 2 * kPBytes;
+  static constexpr int kUsed = kOffRing + kRing * kKVBytes;
   static constexpr int kDynBytes = kUsed + 1024;  // + alignment slack for the 1024-byte swizzle atoms
 };
 
@@ -97,7 +124,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sQ = smem + LY::kOffQ;
   uint8_t *sRing = smem + LY::kOffRing;
-  uint8_t *sP = smem + LY::kOffP;
 
   const int h = blockIdx.x;
   const int qb = n_blocks - 1 - static_cast<int>(blockIdx.y);  // longest rows first
@@ -194,7 +220,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
     } else if (warp == 9 && lane == 0) {
       // ------------------------------ MMA issuer ------------------------------
-      const uint32_t aQ = smem_u32(sQ), aR = smem_u32(sRing), aP = smem_u32(sP);
+      const uint32_t aQ = smem_u32(sQ), aR = smem_u32(sRing);
       int cnt_pv[2] = {0, 0};
       bool ok = mbar_wait(&q_full, 0, &s_abort);
       auto item_ready = [&](int i) -> bool {
@@ -211,15 +237,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         umma_commit(&s_full[w]);
       };
-      auto issue_pv = [&](int w, int j) -> bool {  // O_w += P_w V_j (V_j is item 2j+1)
+      auto issue_pv = [&](int w, int j) -> bool {  // O_w += P_w V_j (V_j is item 2j+1, P_w in TMEM)
         if (!mbar_wait(&p_full[w], cnt_pv[w] & 1, &s_abort)) return false;
         tc_fence_after();
         const uint32_t vb = aR + ((2 * j + 1) % kRing) * LY::kKVBytes;
-        const uint32_t pb = aP + w * LY::kPBytes;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
-          umma_bf16(tmem + 256 + w * D, sw128_desc(pb + (kk >> 2) * (kBM * 128) + (kk & 3) * 32, 16, 1024),
-                    sw128_desc(vb + kk * (16 * 128), kBN * 128, 1024), IDESC_O, (cnt_pv[w] > 0 || kk > 0));
+          umma_bf16_ts(tmem + 256 + w * D, tmem + w * kBN + kk * 8, sw128_desc(vb + kk * (16 * 128), kBN * 128, 1024),
+                       IDESC_O, (cnt_pv[w] > 0 || kk > 0));
         }
         umma_commit(&o_done[w]);
         ++cnt_pv[w];
@@ -268,11 +293,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_off + w * kBN;
     const uint32_t tO = tmem + lane_off + 256 + w * D;
-    uint8_t *myP = sP + w * LY::kPBytes;
+    const uint64_t scale2 = f2pack(scale_log2, scale_log2);
     float m_used = -INFINITY, lsum = 0.f;
     int cnt = 0;
     bool ok = true;
     for (int j = lo[w]; j <= hi[w]; ++j, ++cnt) {
+      // S_w(j) complete also means PV_w(j-1) complete (a commit tracks every earlier
+      // MMA), so O_w may be rescaled and P_w overwritten below.
       if (!__all_sync(0xffffffffu, mbar_wait(&s_full[w], cnt & 1, &s_abort))) {
         ok = false;
         break;
@@ -295,19 +322,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             if (!allowed) sr[c][i] = __float_as_uint(-INFINITY);
           }
       }
-      // row max of the raw scores: 8 independent chains, then a tree
+      // row max of the raw scores: 8 chains of 3-input max, then a tree
       float mx[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mx[k] = __uint_as_float(sr[k >> 2][(k & 3) * 8]);
+      for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < kBN / 32; ++c)
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int e = c * 32 + i, k = (e >> 3) & 7;
-          mx[k] = fmaxf(mx[k], __uint_as_float(sr[c][i]));
-        }
-      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * scale_log2;
+      for (int q = 0; q < kBN / 2; ++q)
+        mx[q & 7] = fmax3(mx[q & 7], __uint_as_float(sr[q >> 4][(2 * q) & 31]),
+                          __uint_as_float(sr[q >> 4][(2 * q + 1) & 31]));
+      const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) *
+                       scale_log2;
       const bool resc = mt > m_used + kRescaleLog2;  // false while the row has seen nothing
       float alpha = 1.f;
       if (resc) {
@@ -315,53 +339,46 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         m_used = mt;
       }
       const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
-      float sm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      const uint64_t negm2 = f2pack(neg_m, neg_m);
+      // P = 2^(s*scale - m), truncated to bf16 (the upper 16 bits, packed two per
+      // column); the row sum adds the same truncated values, so the normalisation
+      // matches what the tensor core multiplies.
+      uint64_t sm2[4] = {0, 0, 0, 0};
+      uint32_t pk[kBN / 2];
 #pragma unroll
-      for (int c = 0; c < kBN / 32; ++c)
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int e = c * 32 + i, k = (e >> 3) & 7;
-          const float p = ex2(fmaf(__uint_as_float(sr[c][i]), scale_log2, neg_m));
-          sm[k] += p;
-          sr[c][i] = __float_as_uint(p);
-        }
-      lsum = lsum * alpha + (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
+      for (int q = 0; q < kBN / 2; ++q) {
+        float x0, x1;
+        f2unpack(ffma2(f2pack(__uint_as_float(sr[q >> 4][(2 * q) & 31]), __uint_as_float(sr[q >> 4][(2 * q + 1) & 31])),
+                       scale2, negm2),
+                 x0, x1);
+        const bool poly = kPolyEvery > 0 && q % kPolyEvery == kPolyEvery - 1;
+        const uint32_t b0 = __float_as_uint(poly ? exp2_poly(x0) : ex2(x0));
+        const uint32_t b1 = __float_as_uint(poly ? exp2_poly(x1) : ex2(x1));
+        pk[q] = __byte_perm(b0, b1, 0x7632);
+        sm2[q & 3] = fadd2(sm2[q & 3], f2pack(__uint_as_float(b0 & 0xFFFF0000u), __uint_as_float(b1 & 0xFFFF0000u)));
+      }
+      float s0, s1, s2, s3, s4, s5, s6, s7;
+      f2unpack(sm2[0], s0, s1);
+      f2unpack(sm2[1], s2, s3);
+      f2unpack(sm2[2], s4, s5);
+      f2unpack(sm2[3], s6, s7);
+      lsum = lsum * alpha + (((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7)));
 
-      // P_j overwrites P_{j-1} and O is rescaled: both wait for PV_{j-1}
-      if (cnt > 0) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&o_done[w], (cnt - 1) & 1, &s_abort))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, resc)) {
+      if (cnt > 0 && __any_sync(0xffffffffu, resc)) {
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t orr[32];
-            tmem_ld32(tO + c * 32, orr);
-            tmem_wait_ld();
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t orr[32];
+          tmem_ld32(tO + c * 32, orr);
+          tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
-            tmem_st32(tO + c * 32, orr);
-          }
-          tmem_wait_st();
+          for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
+          tmem_st32(tO + c * 32, orr);
         }
       }
-      // P row -> shared memory, 128-byte swizzle: 16-byte chunk c of row r at c ^ (r % 8)
-#pragma unroll
-      for (int kb = 0; kb < kBN / 64; ++kb) {
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const int e = kb * 64 + c * 8;
-          uint4 u;
-          u.x = f2_to_bf2(__uint_as_float(sr[e / 32][e % 32 + 0]), __uint_as_float(sr[e / 32][e % 32 + 1]));
-          u.y = f2_to_bf2(__uint_as_float(sr[e / 32][e % 32 + 2]), __uint_as_float(sr[e / 32][e % 32 + 3]));
-          u.z = f2_to_bf2(__uint_as_float(sr[e / 32][e % 32 + 4]), __uint_as_float(sr[e / 32][e % 32 + 5]));
-          u.w = f2_to_bf2(__uint_as_float(sr[e / 32][e % 32 + 6]), __uint_as_float(sr[e / 32][e % 32 + 7]));
-          *reinterpret_cast<uint4 *>(myP + kb * (kBM * 128) + row * 128 + ((c ^ (row & 7)) * 16)) = u;
-        }
-      }
-      fence_proxy_async_smem();
+      // P_w(j) -> the first 64 columns of S_w
+      tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
+      tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[w]);
     }
