@@ -30,7 +30,13 @@ struct DecodePlan {
   int n_splits;
 };
 DecodePlan plan_decode(int B, int G, int n_max, int num_splits);
-constexpr int kDecodeTile = 32;  // keys per pipeline stage
+constexpr int kDecodeTile = 32;     // keys per pipeline stage, one query head per key/value head
+constexpr int kDecodeGqaTile = 64;  // keys per pipeline stage, several query heads per key/value head
+constexpr int kDecodeGrain = 64;    // split chunks are multiples of this many keys
+constexpr int kDecodeMaxGroup = 16; // query heads per key/value head the decode kernels accept
+// The grouped-query decode (H/G > 1) reads 128-byte-swizzled 64x64 tiles; the
+// one-head decode reads unswizzled d x 32 tiles.
+inline bool decode_uses_mma(int H, int G) { return H / G > 1; }
 
 cudaError_t launch_attn_decode(const CUtensorMap &tmK, const CUtensorMap &tmV, const void *q, int H,
                                const olmo3_kv_cache &c, const int32_t *kv_len, const DecodePlan &plan, void *out,

@@ -157,7 +157,7 @@ int olmo3_attn_decode(const void *q, int H, const olmo3_kv_cache *c, const int32
   int st = validate_cache(c);
   if (st != OLMO3_OK) return st;
   if (H < 1 || max_kv_len < 1 || num_splits < 0 || !isfinite(scale)) return OLMO3_ERR_INVALID_ARG;
-  if (H % c->G != 0 || H / c->G > 8) return OLMO3_ERR_UNSUPPORTED;
+  if (H % c->G != 0 || H / c->G > kDecodeMaxGroup) return OLMO3_ERR_UNSUPPORTED;
   if (c->B > 65535) return OLMO3_ERR_UNSUPPORTED;
   if (c->B == 0) return OLMO3_OK;
   if (!q || !kv_len || !out || !aligned16(q) || !aligned16(out)) return OLMO3_ERR_INVALID_ARG;
@@ -170,9 +170,12 @@ int olmo3_attn_decode(const void *q, int H, const olmo3_kv_cache *c, const int32
   CUtensorMap tmK, tmV;
   const cuuint64_t dims[3] = {(cuuint64_t)c->d, (cuuint64_t)c->G, (cuuint64_t)c->total_slots};
   const cuuint64_t strides[2] = {(cuuint64_t)c->d * 2, (cuuint64_t)c->G * c->d * 2};
-  const cuuint32_t box[3] = {(cuuint32_t)c->d, 1, (cuuint32_t)kDecodeTile};
-  if (!encode_bf16(&tmK, c->k, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !encode_bf16(&tmV, c->v, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+  const bool mma = decode_uses_mma(H, c->G);
+  const cuuint32_t box_one[3] = {(cuuint32_t)c->d, 1, (cuuint32_t)kDecodeTile};
+  const cuuint32_t box_mma[3] = {64, 1, (cuuint32_t)kDecodeGqaTile};
+  const CUtensorMapSwizzle swz = mma ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
+  if (!encode_bf16(&tmK, c->k, 3, dims, strides, mma ? box_mma : box_one, swz) ||
+      !encode_bf16(&tmV, c->v, 3, dims, strides, mma ? box_mma : box_one, swz))
     return OLMO3_ERR_CUDA;
   return cuda_status(launch_attn_decode(tmK, tmV, q, H, *c, kv_len, pl, out, lse_out, scale,
                                         static_cast<float *>(workspace), err_dev, as_stream(stream)));

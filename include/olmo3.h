@@ -47,7 +47,7 @@ extern "C" {
 /* ---- status codes ------------------------------------------------------ */
 #define OLMO3_OK               0
 #define OLMO3_ERR_INVALID_ARG (-1)  /* null pointer, negative size, bad enum, misalignment */
-#define OLMO3_ERR_UNSUPPORTED (-2)  /* d not in {64,128}, H % G != 0, H/G > 8, too-wide rows */
+#define OLMO3_ERR_UNSUPPORTED (-2)  /* d not in {64,128}, H % G != 0, H/G > 16, too-wide rows */
 #define OLMO3_ERR_WORKSPACE   (-3)  /* workspace missing or smaller than required */
 #define OLMO3_ERR_CUDA        (-4)  /* a CUDA runtime call or launch failed */
 

@@ -140,8 +140,8 @@ def test_decode_workspace_and_validation(lib):
     c = _cache(layer_type=L.FULL, capacity=16)
     # workspace too small
     assert dec(FAKE, 4, ctypes.byref(c), FAKE, 16, FAKE, NULL, 0.1, 0, FAKE, 4, NULL, NULL) == L.ERR_WORKSPACE
-    # GQA ratio above 8 unsupported
-    assert dec(FAKE, 18, ctypes.byref(c), FAKE, 16, FAKE, NULL, 0.1, 0, FAKE, 1 << 20, NULL, NULL) == \
+    # more than 16 query heads per key/value head unsupported
+    assert dec(FAKE, 34, ctypes.byref(c), FAKE, 16, FAKE, NULL, 0.1, 0, FAKE, 1 << 20, NULL, NULL) == \
         L.ERR_UNSUPPORTED
     assert dec(FAKE, 4, ctypes.byref(c), FAKE, 0, FAKE, NULL, 0.1, 0, FAKE, 1 << 20, NULL, NULL) == \
         L.ERR_INVALID_ARG

@@ -280,14 +280,17 @@ def _decode_case(B, H, G, d, typ, W, lens, seed, num_splits=0, q_scale=1.0):
     (3, 10, 2, 128, 4096, [1000, 33, 4097]),
     (2, 8, 1, 128, 64, [100, 64]),
     (4, 6, 2, 64, 128, [1, 2, 127, 300]),
+    (2, 32, 2, 128, 4096, [70000, 4100]),        # 16 query heads per key/value head
+    (3, 40, 8, 128, 4096, [65537, 64, 65]),      # 32B shapes across a 64-key tile edge
 ])
 def test_decode_parity(typ, B, H, G, d, W, lens):
     _decode_case(B, H, G, d, typ, W, lens, seed=400 + sum(lens))
 
 
 @pytest.mark.parametrize("splits", [1, 3, 7, 200])
-def test_decode_split_count_does_not_change_the_result(splits):
-    _decode_case(3, 4, 4, 128, L.FULL, 4096, [5000, 1, 777], seed=9, num_splits=splits, q_scale=3.0)
+@pytest.mark.parametrize("H,G", [(4, 4), (10, 2)])
+def test_decode_split_count_does_not_change_the_result(splits, H, G):
+    _decode_case(3, H, G, 128, L.FULL, 4096, [5000, 1, 777], seed=9, num_splits=splits, q_scale=3.0)
 
 
 def test_decode_bad_kv_len_sets_error_and_zeroes_only_that_sequence():
