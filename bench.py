@@ -53,6 +53,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--batch", type=int, default=0, help="override B of a decode workload (small profiling captures)")
+    ap.add_argument("--shared-caches", action="store_true",
+                    help="decode: one cache per layer type even when per-layer caches would fit")
     return ap.parse_args()
 
 
@@ -283,7 +285,7 @@ class PrefillStep:
 class DecodeStep:
     """One decode token per sequence through every layer of the model pattern."""
 
-    def __init__(self, name, dev, stream, batch=0):
+    def __init__(self, name, dev, stream, batch=0, shared=False):
         from hybrid_sliding_window_olmo3_b200 import olmo3 as L
         from hybrid_sliding_window_olmo3_b200 import workloads as WL
         self.L = L
@@ -303,7 +305,7 @@ class DecodeStep:
         per_layer = {L.SLIDING: B * W * G * d * 4, L.FULL: B * cap_full * G * d * 4}
         need = sum(per_layer[t] for t in self.types)
         free = torch.cuda.mem_get_info(dev)[0]
-        self.shared = need > 0.8 * free
+        self.shared = shared or need > 0.8 * free
         caches = {}
 
         def make(typ, key):
@@ -435,8 +437,10 @@ class DecodeStep:
                           f"one sliding and one full layer), {el:.1f} s of oracle time; numpy, single thread"}
 
 
-def make_workload(name, dev, stream, batch=0):
-    return PrefillStep(name, dev, stream) if name.endswith("prefill") else DecodeStep(name, dev, stream, batch)
+def make_workload(name, dev, stream, batch=0, shared=False):
+    if name.endswith("prefill"):
+        return PrefillStep(name, dev, stream)
+    return DecodeStep(name, dev, stream, batch, shared)
 
 
 # --------------------------------------------------------------------------
@@ -451,7 +455,7 @@ def run_ours(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
     stream = torch.cuda.current_stream(dev)
-    wk = make_workload(args.workload, dev, stream, args.batch)
+    wk = make_workload(args.workload, dev, stream, args.batch, args.shared_caches)
     peaks, peak_src = load_peaks()
 
     def barrier():
@@ -538,7 +542,7 @@ def run_reference(args):
     if dev is None:
         print(json.dumps({"impl": "reference", "unavailable": "the sampled workload is generated on a CUDA device"}))
         return
-    wk = make_workload(args.workload, dev, torch.cuda.current_stream(dev), args.batch)
+    wk = make_workload(args.workload, dev, torch.cuda.current_stream(dev), args.batch, args.shared_caches)
     per = []
     for i in range(args.warmup + args.steps):
         cb = wk.cpu_baseline(max(2.0, min(8.0, 150.0 / (args.warmup + args.steps))))
