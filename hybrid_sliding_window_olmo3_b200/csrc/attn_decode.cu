@@ -317,7 +317,10 @@ __global__ void __launch_bounds__(D) attn_decode_combine_kernel(const int32_t *_
 // ldmatrix.trans.  The partials use the same workspace layout and combine as the
 // one-head kernel.
 // ---------------------------------------------------------------------------
-constexpr int kGqaStages = 3;
+#ifndef OLMO3_GQA_STAGES
+#define OLMO3_GQA_STAGES 3
+#endif
+constexpr int kGqaStages = OLMO3_GQA_STAGES;
 constexpr int kGqaWarps = 4;  // compute warps; one more warp produces
 constexpr int kGqaThreads = (kGqaWarps + 1) * 32;
 
@@ -579,24 +582,28 @@ __global__ void __launch_bounds__(kGqaThreads) attn_decode_gqa_kernel(
   }
 }
 
-DecodePlan plan_decode(int B, int G, int n_max, int num_splits) {
+DecodePlan plan_decode(int B, int G, int n_max, int num_splits, bool mma) {
   DecodePlan pl;
-  const int64_t tiles = (static_cast<int64_t>(n_max) + kDecodeGrain - 1) / kDecodeGrain;
+  const int64_t grains = (static_cast<int64_t>(n_max) + kDecodeGrain - 1) / kDecodeGrain;
   int64_t splits;
   if (num_splits > 0) {
     splits = num_splits;
   } else {
-    // aim at >= 8 waves of 3 CTAs per SM on 148 SMs, with at least 2 grains (128 keys) per CTA
-    const int64_t target = 148 * 3 * 8;
+    // Enough CTAs for several waves of the resident CTAs (3 per SM for the one-head
+    // kernel, 2 for the grouped-query kernel, whose stages are larger), but at
+    // least 1024 keys per split: short splits spend their time filling the pipeline
+    // (measured on the 32B sliding layer: 4 splits of 1024 keys take 27 us, 32 splits
+    // of 128 keys 47 us).
+    const int64_t target = mma ? 148 * 2 * 4 : 148 * 3 * 8;
     const int64_t pairs = static_cast<int64_t>(B) * G;
     splits = (target + pairs - 1) / pairs;
-    const int64_t max_splits = (tiles + 1) / 2;
+    const int64_t max_splits = (grains + 15) / 16;
     if (splits > max_splits) splits = max_splits;
   }
   if (splits < 1) splits = 1;
-  if (splits > tiles) splits = tiles;
-  const int64_t tiles_per_split = (tiles + splits - 1) / splits;
-  pl.chunk = static_cast<int>(tiles_per_split * kDecodeGrain);
+  if (splits > grains) splits = grains;
+  const int64_t grains_per_split = (grains + splits - 1) / splits;
+  pl.chunk = static_cast<int>(grains_per_split * kDecodeGrain);
   pl.n_splits = static_cast<int>((n_max + static_cast<int64_t>(pl.chunk) - 1) / pl.chunk);
   return pl;
 }

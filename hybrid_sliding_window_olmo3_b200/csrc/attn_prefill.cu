@@ -46,36 +46,15 @@ constexpr float kRescaleLog2 = 8.0f;
 #ifndef OLMO3_PF_CONTROL_REGS
 #define OLMO3_PF_CONTROL_REGS 64
 #endif
-#ifndef OLMO3_PF_EXP2_POLY_EVERY
-#define OLMO3_PF_EXP2_POLY_EVERY 0
-#endif
 // Register split between the control warpgroup and the two softmax warpgroups:
 // 128 x control + 256 x softmax must not exceed 384 x 168 (the launch budget).
 constexpr uint32_t kControlRegs = OLMO3_PF_CONTROL_REGS;
 constexpr uint32_t kSoftmaxRegs = ((384u * 168u - 128u * kControlRegs) / 256u) & ~7u;
-// Every kPolyEvery-th score of a row takes its exp2 on the FMA pipe (exp2_poly)
-// instead of the transcendental unit, which the rest of the exps saturate.
-constexpr int kPolyEvery = OLMO3_PF_EXP2_POLY_EVERY;
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// 2^x on the FMA and integer pipes.  Cody-Waite style range reduction x = j + f
-// with j = round(x) (adding and removing 1.5 * 2^23 rounds to an integer held in
-// the low mantissa bits) and |f| <= 1/2, then a degree-3 polynomial for 2^f whose
-// coefficients are a Remez (minimax relative error) fit on [-1/2, 1/2], max
-// relative error 7.5e-5 (far below the 2^-8 of the bf16 P it feeds); j is added
-// to the exponent field.  x is clamped to >= -126 so the result stays >= 0
-// (2^-126 stands for the exp of a masked score, i.e. 0 at bf16 precision).
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  const float p = fmaf(fmaf(fmaf(0.0551716685f, f, 0.242611125f), f, 0.693260968f), f, 0.999928057f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 template <uint32_t N>
@@ -351,9 +330,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         f2unpack(ffma2(f2pack(__uint_as_float(sr[q >> 4][(2 * q) & 31]), __uint_as_float(sr[q >> 4][(2 * q + 1) & 31])),
                        scale2, negm2),
                  x0, x1);
-        const bool poly = kPolyEvery > 0 && q % kPolyEvery == kPolyEvery - 1;
-        const uint32_t b0 = __float_as_uint(poly ? exp2_poly(x0) : ex2(x0));
-        const uint32_t b1 = __float_as_uint(poly ? exp2_poly(x1) : ex2(x1));
+        const uint32_t b0 = __float_as_uint(ex2(x0));
+        const uint32_t b1 = __float_as_uint(ex2(x1));
         pk[q] = __byte_perm(b0, b1, 0x7632);
         sm2[q & 3] = fadd2(sm2[q & 3], f2pack(__uint_as_float(b0 & 0xFFFF0000u), __uint_as_float(b1 & 0xFFFF0000u)));
       }

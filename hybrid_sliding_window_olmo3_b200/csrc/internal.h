@@ -29,7 +29,7 @@ struct DecodePlan {
   int chunk;
   int n_splits;
 };
-DecodePlan plan_decode(int B, int G, int n_max, int num_splits);
+DecodePlan plan_decode(int B, int G, int n_max, int num_splits, bool mma);
 constexpr int kDecodeTile = 32;     // keys per pipeline stage, one query head per key/value head
 constexpr int kDecodeGqaTile = 64;  // keys per pipeline stage, several query heads per key/value head
 constexpr int kDecodeGrain = 64;    // split chunks are multiples of this many keys

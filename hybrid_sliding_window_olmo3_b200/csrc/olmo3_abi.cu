@@ -147,7 +147,7 @@ size_t olmo3_attn_decode_workspace_size(int B, int H, int G, int d, int max_kv_l
       window < 1 || num_splits < 0)
     return 0;
   const int n_max = layer_type == OLMO3_SLIDING ? (max_kv_len < window ? max_kv_len : window) : max_kv_len;
-  const DecodePlan pl = plan_decode(B, G, n_max, num_splits);
+  const DecodePlan pl = plan_decode(B, G, n_max, num_splits, decode_uses_mma(H, G));
   return static_cast<size_t>(B) * H * pl.n_splits * (d + 2) * sizeof(float);
 }
 
@@ -165,7 +165,7 @@ int olmo3_attn_decode(const void *q, int H, const olmo3_kv_cache *c, const int32
       olmo3_attn_decode_workspace_size(c->B, H, c->G, c->d, max_kv_len, c->layer_type, c->window, num_splits);
   if (workspace == nullptr || ws_bytes < need || !aligned16(workspace)) return OLMO3_ERR_WORKSPACE;
   const int n_max = c->layer_type == OLMO3_SLIDING ? (max_kv_len < c->window ? max_kv_len : c->window) : max_kv_len;
-  const DecodePlan pl = plan_decode(c->B, c->G, n_max, num_splits);
+  const DecodePlan pl = plan_decode(c->B, c->G, n_max, num_splits, decode_uses_mma(H, c->G));
   if (pl.n_splits > 65535) return OLMO3_ERR_UNSUPPORTED;
   CUtensorMap tmK, tmV;
   const cuuint64_t dims[3] = {(cuuint64_t)c->d, (cuuint64_t)c->G, (cuuint64_t)c->total_slots};
