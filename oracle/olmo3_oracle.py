@@ -48,7 +48,7 @@ __all__ = [
     "SLIDING", "FULL", "layer_types", "sliding_window_mask", "causal_mask",
     "attention_masks", "allowed", "allowed_count", "rms_norm", "rope_inv_freq",
     "rope", "qk_norm_rope", "attend", "prefill_attention", "KVCache",
-    "append_slots", "decode_attention", "full_recompute_last_row",
+    "append_slots", "decode_attention", "full_recompute_last_row", "chunk_attention",
     "kv_bytes_per_token", "kv_cache_bytes",
 ]
 
@@ -283,6 +283,31 @@ def decode_attention(q_hat, caches, q_pos, layer_type: str, window: int,
                         scale, k_valid=c.valid()[None])
         outs.append(o[0, 0])
         lses.append(lse[0, :, 0])
+    return np.stack(outs), np.stack(lses)
+
+
+def chunk_attention(q_hat, k_hat, v, caches, pos_offset, layer_type: str, window: int,
+                    scale: float | None = None):
+    """A chunk of T new tokens per sequence (positions pos_offset[b] + t) attends
+    over what its cache holds before the chunk plus the chunk itself.
+
+    q_hat: [B, T, H, d]; k_hat, v: [B, T, G, d] (already normed / rotated);
+    caches: list of B KVCache holding positions < pos_offset[b] (not yet updated).
+    Returns (O [B, T, H, d], lse [B, H, T]).
+    """
+    q_hat = np.asarray(q_hat, dtype=np.float64)
+    B, T = q_hat.shape[:2]
+    outs, lses = [], []
+    for b in range(B):
+        c = caches[b]
+        keep = c.valid()
+        p = int(pos_offset[b]) + np.arange(T)
+        k_all = np.concatenate([c.k[keep], np.asarray(k_hat[b], dtype=np.float64)])[None]
+        v_all = np.concatenate([c.v[keep], np.asarray(v[b], dtype=np.float64)])[None]
+        kp = np.concatenate([c.pos[keep], p])[None]
+        o, lse = attend(q_hat[b][None], p[None], k_all, kp, v_all, layer_type, window, scale)
+        outs.append(o[0])
+        lses.append(lse[0])
     return np.stack(outs), np.stack(lses)
 
 

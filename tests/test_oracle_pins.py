@@ -339,6 +339,28 @@ def test_decode_with_cache_equals_full_recompute(typ):
         np.testing.assert_allclose(o, ref, atol=1e-12)
 
 
+@pytest.mark.parametrize("typ", ["sliding", "full"])
+def test_chunked_prefill_equals_one_shot_prefill(typ):
+    # "Apply RoPE with position offsets for cache compatibility": feeding a prompt in
+    # chunks through the cache must give the rows of the one-shot prefill.
+    rng = np.random.default_rng(12)
+    W, H, G, d, Ttot = 5, 4, 2, 8, 23
+    q = rng.standard_normal((1, Ttot, H, d))
+    k = rng.standard_normal((1, Ttot, G, d))
+    v = rng.standard_normal((1, Ttot, G, d))
+    ref, ref_lse = O.prefill_attention(q, k, v, typ, W)
+    cap = W if typ == "sliding" else Ttot
+    c = O.KVCache(typ, cap, G, d)
+    p0 = 0
+    for T in (1, 4, 7, 2, 9):
+        o, lse = O.chunk_attention(q[:, p0:p0 + T], k[:, p0:p0 + T], v[:, p0:p0 + T], [c], [p0], typ, W)
+        np.testing.assert_allclose(o, ref[:, p0:p0 + T], atol=1e-12)
+        np.testing.assert_allclose(lse, ref_lse[:, :, p0:p0 + T], atol=1e-12)
+        c.append(range(p0, p0 + T), k[0, p0:p0 + T], v[0, p0:p0 + T])
+        p0 += T
+    assert p0 == Ttot
+
+
 def test_kv_sizing_matches_the_pages():
     g = {r[0]: float(r[1]) for r in read_golden("kv_sizing.txt")}
     t32 = O.layer_types(32)
