@@ -208,14 +208,15 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(
 #pragma unroll
       for (int it = 0; it < NIT; ++it) {
         const int kk = warp * KEYS_PER_WARP + it * KPW + lg;
+        const bool valid = key_base + kk < k_end;  // a partly used tile may hold uninitialised rows
         const uint4 u = *reinterpret_cast<const uint4 *>(vt + kk * D + li * 8);
         const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
         float vf[8];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const float2 f = bf2_to_f2(w4[j]);
-          vf[2 * j] = f.x;
-          vf[2 * j + 1] = f.y;
+          vf[2 * j] = valid ? f.x : 0.f;
+          vf[2 * j + 1] = valid ? f.y : 0.f;
         }
 #pragma unroll
         for (int r = 0; r < R; ++r)
@@ -511,6 +512,19 @@ __global__ void __launch_bounds__(kGqaThreads) attn_decode_gqa_kernel(
         o[nb][2] *= a_hi;
         o[nb][3] *= a_hi;
       }
+      // V rows past the last key of a partly used tile may be uninitialised cache
+      // slots: zero this warp's share of them (P is 0 there, but 0 x NaN is not 0)
+      const int tile_key0 = k_begin + i * kDecodeGqaTile;
+      if (tile_key0 + kDecodeGqaTile > k_end) {
+        uint8_t *vt = sV + st * S::kTileBytes;
+        for (int e = lane; e < 16 * NDB * 8; e += 32) {
+          const int r = e / (NDB * 8), db = (e / 8) % NDB, c = e % 8;
+          const int key = warp * 16 + r;
+          if (tile_key0 + key >= k_end)
+            *reinterpret_cast<uint4 *>(vt + db * (kDecodeGqaTile * 128) + key * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+        }
+        __syncwarp();
+      }
       // P (16 rows x 16 keys) as the A operand, straight from the S fragments
       const uint32_t pa[4] = {f2_to_bf2(p[0][0], p[0][1]), f2_to_bf2(p[0][2], p[0][3]), f2_to_bf2(p[1][0], p[1][1]),
                               f2_to_bf2(p[1][2], p[1][3])};
@@ -524,6 +538,7 @@ __global__ void __launch_bounds__(kGqaThreads) attn_decode_gqa_kernel(
         mma_16816(o[2 * nb2], pa, b0, b1);
         mma_16816(o[2 * nb2 + 1], pa, b2, b3);
       }
+      if (tile_key0 + kDecodeGqaTile > k_end) fence_proxy_async_smem();  // before TMA refills what we zeroed
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty_bar[st]);
     }

@@ -76,19 +76,31 @@ struct PfLayout {
   static constexpr int kDynBytes = kUsed + 1024;  // + alignment slack for the 1024-byte swizzle atoms
 };
 
-// Tiles (in units of kBN keys) a query tile [r0, r1] needs: [first, last].
-__device__ __forceinline__ void band_tiles(int r0, int r1, bool is_full, int window, int &first, int &last) {
-  const int64_t lo = static_cast<int64_t>(r0) - window + 1;
-  first = (is_full || lo < 0) ? 0 : static_cast<int>(lo / kBN);
-  last = r1 / kBN;
+// Key tiles (in units of kBN keys of the key rows) that query rows at absolute
+// positions [t0, t1] need, when key row j holds absolute position kp0 + j and
+// rows 0 .. klen-1 exist: [first, last], empty when last < first.
+__device__ __forceinline__ void band_tiles(int t0, int t1, int kp0, int klen, bool is_full, int window,
+                                           int &first, int &last) {
+  const int64_t w_lo = static_cast<int64_t>(t0) - window + 1;
+  const int64_t lo_abs = (is_full || w_lo < kp0) ? static_cast<int64_t>(kp0) : w_lo;
+  const int64_t k_hi = static_cast<int64_t>(kp0) + klen - 1;
+  const int64_t hi_abs = t1 < k_hi ? static_cast<int64_t>(t1) : k_hi;
+  if (hi_abs < lo_abs) {
+    first = 1;
+    last = 0;
+    return;
+  }
+  first = static_cast<int>((lo_abs - kp0) / kBN);
+  last = static_cast<int>((hi_abs - kp0) / kBN);
 }
 
-template <int D>
+template <int D, int MODE>
 __global__ void __launch_bounds__(kPfThreads, 1)
     attn_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, __nv_bfloat16 *__restrict__ out,
-                        float *__restrict__ lse_out, int T, int H, int G, int layer_type, int window,
-                        float scale_log2, int n_blocks, int *err) {
+                        float *__restrict__ lse_out, int Tq, int Tk, int H, int G, int layer_type, int window,
+                        float scale_log2, int n_blocks, const int32_t *__restrict__ pos_offset,
+                        const int64_t *__restrict__ seq_base, int *err) {
   using LY = PfLayout<D>;
   constexpr int NDB = D / 64;  // 64-feature (128-byte) blocks per row
   constexpr uint32_t IDESC_S = idesc_bf16_f32(kBM, kBN, 0);
@@ -111,22 +123,40 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const int q0 = qb * 2 * kBM;
   const bool is_full = layer_type == OLMO3_FULL;
 
+  // Positions.  Query row t (0 <= t < Tq) sits at absolute position qp0 + t; key
+  // row j (0 <= j < klen) is row krow0 + j of the K/V tensor maps and sits at
+  // absolute position kp0 + j.
+  //   kPrefillFresh   a fresh sequence: qp0 = kp0 = 0, keys are the sequence itself.
+  //   kPrefillCache   a chunk at pos_offset[b] over a linear cache that already holds
+  //                   it: keys are cache rows seq_base[b] + j, positions 0 .. qp0+Tq-1.
+  //   kPrefillWindow  a chunk at pos_offset[b] over a gathered window: rows b*Tk + j
+  //                   hold positions max(0, qp0 - window + 1) .. qp0 + Tq - 1.
+  // MODE is a template parameter so that the fresh-sequence kernel carries none
+  // of the offset arithmetic (it costs registers in the softmax loop).
+  int qp0 = 0, kp0 = 0, klen = Tk;
+  int64_t krow0 = static_cast<int64_t>(b) * Tk;
+  if (MODE != kPrefillFresh) qp0 = pos_offset[b];
+  if (MODE == kPrefillCache) {
+    krow0 = seq_base[b];
+    klen = qp0 + Tq;
+  } else if (MODE == kPrefillWindow) {
+    kp0 = max(0, qp0 - window + 1);
+    klen = qp0 + Tq - kp0;
+  }
+
   // key-tile ranges: the union [kt_lo, kt_lo + n_kt) and, per query tile w, [lo_w, hi_w] inside it
   int lo[2], hi[2];
 #pragma unroll
   for (int w = 0; w < 2; ++w) {
     const int r0 = q0 + w * kBM;
-    if (r0 < T) {
-      int f, l;
-      band_tiles(r0, min(r0 + kBM, T) - 1, is_full, window, f, l);
-      lo[w] = f;
-      hi[w] = l;
+    if (r0 < Tq) {
+      band_tiles(qp0 + r0, qp0 + min(r0 + kBM, Tq) - 1, kp0, klen, is_full, window, lo[w], hi[w]);
     } else {
       lo[w] = 1;
       hi[w] = 0;  // empty: every row of this tile is past the sequence
     }
   }
-  const int kt_lo = lo[0];
+  const int kt_lo = hi[0] >= lo[0] ? lo[0] : lo[1];
   const int kt_hi = hi[1] >= lo[1] ? hi[1] : hi[0];
   const int n_kt = kt_hi - kt_lo + 1;
 #pragma unroll
@@ -182,12 +212,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           ok = false;
           break;
         }
-        const int k0 = (kt_lo + (i >> 1)) * kBN;
+        const int krow = static_cast<int>(krow0 + static_cast<int64_t>(kt_lo + (i >> 1)) * kBN);
         const CUtensorMap *tm = (i & 1) ? &tmV : &tmK;
         mbar_arrive_expect_tx(&ring_full[slot], LY::kKVBytes);
 #pragma unroll
         for (int db = 0; db < NDB; ++db)
-          tma_load_4d(sRing + slot * LY::kKVBytes + db * kBN * 128, tm, &ring_full[slot], db * 64, g, k0, b);
+          tma_load_3d(sRing + slot * LY::kKVBytes + db * kBN * 128, tm, &ring_full[slot], db * 64, g, krow);
         ++issued;
       }
       if (!ok) {
@@ -231,6 +261,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       };
       auto active = [&](int w, int j) { return lo[w] <= j && j <= hi[w]; };
 
+      if (n_kt <= 0) ok = false;  // cannot happen for a valid call: every row sees at least its own key
       if (ok) ok = item_ready(0);
       if (ok) {
         tc_fence_after();
@@ -268,7 +299,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int w = warp >> 2;            // query tile of this warpgroup
     const int row = threadIdx.x & 127;  // TMEM lane and row inside the tile
     const int r0 = q0 + w * kBM;
-    const int t = r0 + row;
+    const int t = r0 + row;            // query row
+    const int ta0 = qp0 + r0;          // absolute position of the tile's first row
+    const int ta = qp0 + t;            // absolute position of this row
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_off + w * kBN;
     const uint32_t tO = tmem + lane_off + 256 + w * D;
@@ -289,15 +322,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       for (int c = 0; c < kBN / 32; ++c) tmem_ld32(tS + c * 32, sr[c]);
       tmem_wait_ld();
 
-      const int k0 = (kt_lo + j) * kBN;
-      const bool need_mask = !(k0 + kBN - 1 <= r0 && (is_full || (r0 + kBM - 1) - k0 < window));
+      const int k0 = (kt_lo + j) * kBN;  // key row of the tile's first column
+      const int ka0 = kp0 + k0;           // its absolute position
+      const bool need_mask = !(ka0 + kBN - 1 <= ta0 && (is_full || (ta0 + kBM - 1) - ka0 < window) &&
+                               (MODE == kPrefillFresh || k0 + kBN <= klen));
       if (need_mask) {
 #pragma unroll
         for (int c = 0; c < kBN / 32; ++c)
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const int key = k0 + c * 32 + i;
-            const bool allowed = key <= t && (is_full || t - key < window);
+            const int ka = ka0 + c * 32 + i;
+            const bool allowed = ka <= ta && (is_full || ta - ka < window) &&
+                                 (MODE == kPrefillFresh || k0 + c * 32 + i < klen);
             if (!allowed) sr[c][i] = __float_as_uint(-INFINITY);
           }
       }
@@ -369,13 +405,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     } else if (cnt > 0) {
       tc_fence_after();
       const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-      __nv_bfloat16 *orow = out + ((static_cast<int64_t>(b) * T + t) * H + h) * D;
+      __nv_bfloat16 *orow = out + ((static_cast<int64_t>(b) * Tq + t) * H + h) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t orr[32];
         tmem_ld32(tO + c * 32, orr);
         tmem_wait_ld();
-        if (t < T) {
+        if (t < Tq) {
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
             uint4 u;
@@ -387,9 +423,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
         }
       }
-      if (lse_out != nullptr && t < T) {
+      if (lse_out != nullptr && t < Tq) {
         const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
-        lse_out[(static_cast<int64_t>(b) * H + h) * T + t] = (m_eff + log2f(lsum)) * 0.69314718055994531f;
+        lse_out[(static_cast<int64_t>(b) * H + h) * Tq + t] = (m_eff + log2f(lsum)) * 0.69314718055994531f;
       }
     }
   }
@@ -402,31 +438,54 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   }
 }
 
-template <int D>
+template <int D, int MODE>
 static cudaError_t launch_pf(const CUtensorMap &tmQ, const CUtensorMap &tmK, const CUtensorMap &tmV, void *out,
-                             float *lse_out, int B, int T, int H, int G, int layer_type, int window, float scale,
-                             int *err, cudaStream_t stream) {
+                             float *lse_out, int B, int Tq, int Tk, int H, int G, int layer_type, int window,
+                             float scale, const int32_t *pos_offset, const int64_t *seq_base, int *err,
+                             cudaStream_t stream) {
   using LY = PfLayout<D>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e =
-        cudaFuncSetAttribute(attn_prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::kDynBytes);
+    cudaError_t e = cudaFuncSetAttribute(attn_prefill_kernel<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         LY::kDynBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const int n_blocks = (T + 2 * kBM - 1) / (2 * kBM);
+  const int n_blocks = (Tq + 2 * kBM - 1) / (2 * kBM);
   dim3 grid(H, n_blocks, B);
-  attn_prefill_kernel<D><<<grid, kPfThreads, LY::kDynBytes, stream>>>(
-      tmQ, tmK, tmV, static_cast<__nv_bfloat16 *>(out), lse_out, T, H, G, layer_type, window,
-      scale * 1.4426950408889634f, n_blocks, err);
+  attn_prefill_kernel<D, MODE><<<grid, kPfThreads, LY::kDynBytes, stream>>>(
+      tmQ, tmK, tmV, static_cast<__nv_bfloat16 *>(out), lse_out, Tq, Tk, H, G, layer_type, window,
+      scale * 1.4426950408889634f, n_blocks, pos_offset, seq_base, err);
   return cudaGetLastError();
 }
 
+template <int D>
+static cudaError_t launch_pf_mode(int mode, const CUtensorMap &tmQ, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                                  void *out, float *lse_out, int B, int Tq, int Tk, int H, int G, int layer_type,
+                                  int window, float scale, const int32_t *pos_offset, const int64_t *seq_base,
+                                  int *err, cudaStream_t stream) {
+  switch (mode) {
+    case kPrefillFresh:
+      return launch_pf<D, kPrefillFresh>(tmQ, tmK, tmV, out, lse_out, B, Tq, Tk, H, G, layer_type, window, scale,
+                                         pos_offset, seq_base, err, stream);
+    case kPrefillCache:
+      return launch_pf<D, kPrefillCache>(tmQ, tmK, tmV, out, lse_out, B, Tq, Tk, H, G, layer_type, window, scale,
+                                         pos_offset, seq_base, err, stream);
+    default:
+      return launch_pf<D, kPrefillWindow>(tmQ, tmK, tmV, out, lse_out, B, Tq, Tk, H, G, layer_type, window, scale,
+                                          pos_offset, seq_base, err, stream);
+  }
+}
+
 cudaError_t launch_attn_prefill(const CUtensorMap &tmQ, const CUtensorMap &tmK, const CUtensorMap &tmV, void *out,
-                                float *lse_out, int B, int T, int H, int G, int d, int layer_type, int window,
-                                float scale, int *err, cudaStream_t stream) {
-  if (d == 64) return launch_pf<64>(tmQ, tmK, tmV, out, lse_out, B, T, H, G, layer_type, window, scale, err, stream);
-  return launch_pf<128>(tmQ, tmK, tmV, out, lse_out, B, T, H, G, layer_type, window, scale, err, stream);
+                                float *lse_out, int B, int Tq, int Tk, int H, int G, int d, int layer_type,
+                                int window, float scale, int mode, const int32_t *pos_offset,
+                                const int64_t *seq_base, int *err, cudaStream_t stream) {
+  if (d == 64)
+    return launch_pf_mode<64>(mode, tmQ, tmK, tmV, out, lse_out, B, Tq, Tk, H, G, layer_type, window, scale,
+                              pos_offset, seq_base, err, stream);
+  return launch_pf_mode<128>(mode, tmQ, tmK, tmV, out, lse_out, B, Tq, Tk, H, G, layer_type, window, scale,
+                             pos_offset, seq_base, err, stream);
 }
 
 }  // namespace olmo3

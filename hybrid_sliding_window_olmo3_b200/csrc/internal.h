@@ -45,8 +45,22 @@ cudaError_t launch_attn_decode(const CUtensorMap &tmK, const CUtensorMap &tmV, c
 constexpr int kPrefillBM = 128;  // query rows per CTA
 constexpr int kPrefillBN = 128;  // keys per tile
 
+// Where the keys of a prefill come from (see attn_prefill_kernel).
+constexpr int kPrefillFresh = 0;   // the sequence itself, positions 0 .. T-1
+constexpr int kPrefillCache = 1;   // a linear cache already holding the chunk
+constexpr int kPrefillWindow = 2;  // a gathered window of a ring plus the chunk
+
+// tmK / tmV are 3-d maps over [rows, G, d] with 64 x 1 x 128 boxes (128-byte swizzle).
 cudaError_t launch_attn_prefill(const CUtensorMap &tmQ, const CUtensorMap &tmK, const CUtensorMap &tmV, void *out,
-                                float *lse_out, int B, int T, int H, int G, int d, int layer_type, int window,
-                                float scale, int *err, cudaStream_t stream);
+                                float *lse_out, int B, int Tq, int Tk, int H, int G, int d, int layer_type,
+                                int window, float scale, int mode, const int32_t *pos_offset,
+                                const int64_t *seq_base, int *err, cudaStream_t stream);
+
+// Copies, for each sequence, the window of keys a chunk at pos_offset[b] needs:
+// rows j < Tk of [B, Tk, G, d] hold position max(0, p0 - window + 1) + j, from the
+// ring for positions < p0 and from the chunk after; rows past the chunk are zeroed.
+cudaError_t launch_gather_window(const olmo3_kv_cache &c, const void *k_new, const void *v_new,
+                                 const int32_t *pos_offset, int T, int Tk, void *k_out, void *v_out,
+                                 cudaStream_t stream);
 
 }  // namespace olmo3

@@ -45,6 +45,22 @@ bool encode_bf16(CUtensorMap *tm, const void *base, int rank, const cuuint64_t *
   return r == CUDA_SUCCESS;
 }
 
+// q / out [B, T, H, d] as a 4-d map (query tiles of 128 rows of one head).
+bool encode_q(CUtensorMap *tm, const void *q, int B, int T, int H, int d) {
+  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kPrefillBM), 1};
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)T * H * d * 2};
+  return encode_bf16(tm, q, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// K or V rows [rows, G, d] as a 3-d map (key tiles of 128 rows of one key/value head).
+bool encode_kv(CUtensorMap *tm, const void *base, int64_t rows, int G, int d) {
+  const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(kPrefillBN)};
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)G, (cuuint64_t)rows};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)G * d * 2};
+  return encode_bf16(tm, base, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 int validate_cache(const olmo3_kv_cache *c) {
   if (c == nullptr || c->k == nullptr || c->v == nullptr || c->seq_base == nullptr) return OLMO3_ERR_INVALID_ARG;
   if (!valid_type(c->layer_type) || c->B < 0 || c->G < 1 || c->capacity < 1 || c->total_slots < 1 ||
@@ -124,21 +140,66 @@ int olmo3_attn_prefill(const void *q, const void *k, const void *v, void *out, i
     return OLMO3_ERR_INVALID_ARG;
   if (!valid_d(d) || H % G != 0) return OLMO3_ERR_UNSUPPORTED;
   if (B > 65535 || (T + kPrefillBM - 1) / kPrefillBM > 65535) return OLMO3_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(B) * T >= (int64_t(1) << 31)) return OLMO3_ERR_UNSUPPORTED;
   if (B == 0 || T == 0) return OLMO3_OK;
   if (!q || !k || !v || !out) return OLMO3_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return OLMO3_ERR_INVALID_ARG;
   CUtensorMap tmQ, tmK, tmV;
-  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kPrefillBM), 1};
-  const cuuint64_t dq[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-  const cuuint64_t sq[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)T * H * d * 2};
-  const cuuint64_t dk[4] = {(cuuint64_t)d, (cuuint64_t)G, (cuuint64_t)T, (cuuint64_t)B};
-  const cuuint64_t sk[3] = {(cuuint64_t)d * 2, (cuuint64_t)G * d * 2, (cuuint64_t)T * G * d * 2};
-  if (!encode_bf16(&tmQ, q, 4, dq, sq, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_bf16(&tmK, k, 4, dk, sk, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_bf16(&tmV, v, 4, dk, sk, box, CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!encode_q(&tmQ, q, B, T, H, d) || !encode_kv(&tmK, k, static_cast<int64_t>(B) * T, G, d) ||
+      !encode_kv(&tmV, v, static_cast<int64_t>(B) * T, G, d))
     return OLMO3_ERR_CUDA;
-  return cuda_status(launch_attn_prefill(tmQ, tmK, tmV, out, lse_out, B, T, H, G, d, layer_type, window, scale,
-                                         err_dev, as_stream(stream)));
+  return cuda_status(launch_attn_prefill(tmQ, tmK, tmV, out, lse_out, B, T, T, H, G, d, layer_type, window, scale,
+                                         kPrefillFresh, nullptr, nullptr, err_dev, as_stream(stream)));
+}
+
+size_t olmo3_attn_prefill_chunk_workspace_size(int B, int T, int G, int d, int layer_type, int window) {
+  if (B < 0 || T < 0 || G < 1 || !valid_d(d) || !valid_type(layer_type) || window < 1) return 0;
+  if (layer_type == OLMO3_FULL) return 0;
+  return 2 * static_cast<size_t>(B) * (static_cast<size_t>(window) - 1 + T) * G * d * 2;
+}
+
+int olmo3_attn_prefill_chunk(const void *q, const void *k_new, const void *v_new, const olmo3_kv_cache *c,
+                             const int32_t *pos_offset, int T, int H, void *out, float scale, float *lse_out,
+                             void *workspace, size_t ws_bytes, int *err_dev, void *stream) {
+  int st = validate_cache(c);
+  if (st != OLMO3_OK) return st;
+  if (T < 0 || H < 1 || !isfinite(scale)) return OLMO3_ERR_INVALID_ARG;
+  if (H % c->G != 0) return OLMO3_ERR_UNSUPPORTED;
+  if (c->B > 65535 || (T + kPrefillBM - 1) / kPrefillBM > 65535) return OLMO3_ERR_UNSUPPORTED;
+  if (c->B == 0 || T == 0) return OLMO3_OK;
+  if (!q || !k_new || !v_new || !out || !pos_offset) return OLMO3_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(out)) return OLMO3_ERR_INVALID_ARG;
+  const int B = c->B, G = c->G, d = c->d;
+  const size_t need = olmo3_attn_prefill_chunk_workspace_size(B, T, G, d, c->layer_type, c->window);
+  const int Tk = c->window - 1 + T;
+  if (c->layer_type == OLMO3_SLIDING) {
+    if (workspace == nullptr || ws_bytes < need || !aligned16(workspace)) return OLMO3_ERR_WORKSPACE;
+    if (static_cast<int64_t>(B) * Tk >= (int64_t(1) << 31)) return OLMO3_ERR_UNSUPPORTED;
+  }
+  cudaStream_t s = as_stream(stream);
+  CUtensorMap tmQ, tmK, tmV;
+  if (!encode_q(&tmQ, q, B, T, H, d)) return OLMO3_ERR_CUDA;
+  if (c->layer_type == OLMO3_FULL) {
+    // the chunk goes into the linear cache first (it overwrites nothing), then the
+    // chunk's rows attend over the cache rows 0 .. pos_offset + T - 1
+    if (!encode_kv(&tmK, c->k, c->total_slots, G, d) || !encode_kv(&tmV, c->v, c->total_slots, G, d))
+      return OLMO3_ERR_CUDA;
+    cudaError_t e = launch_kv_append(*c, k_new, v_new, pos_offset, T, nullptr, err_dev, s);
+    if (e != cudaSuccess) return OLMO3_ERR_CUDA;
+    return cuda_status(launch_attn_prefill(tmQ, tmK, tmV, out, lse_out, B, T, 0, H, G, d, OLMO3_FULL, c->window,
+                                           scale, kPrefillCache, pos_offset, c->seq_base, err_dev, s));
+  }
+  // sliding: the ring's window and the chunk are gathered, attended, then the chunk is appended
+  void *wk = workspace;
+  void *wv = static_cast<uint8_t *>(workspace) + need / 2;
+  if (!encode_kv(&tmK, wk, static_cast<int64_t>(B) * Tk, G, d) || !encode_kv(&tmV, wv, static_cast<int64_t>(B) * Tk, G, d))
+    return OLMO3_ERR_CUDA;
+  cudaError_t e = launch_gather_window(*c, k_new, v_new, pos_offset, T, Tk, wk, wv, s);
+  if (e != cudaSuccess) return OLMO3_ERR_CUDA;
+  e = launch_attn_prefill(tmQ, tmK, tmV, out, lse_out, B, T, Tk, H, G, d, OLMO3_SLIDING, c->window, scale,
+                          kPrefillWindow, pos_offset, c->seq_base, err_dev, s);
+  if (e != cudaSuccess) return OLMO3_ERR_CUDA;
+  return cuda_status(launch_kv_append(*c, k_new, v_new, pos_offset, T, nullptr, err_dev, s));
 }
 
 size_t olmo3_attn_decode_workspace_size(int B, int H, int G, int d, int max_kv_len, int layer_type, int window,

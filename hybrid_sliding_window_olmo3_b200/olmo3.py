@@ -280,3 +280,43 @@ def attn_decode_noalloc(q: torch.Tensor, cache: KVCache, kv_len: torch.Tensor, m
     _check("olmo3_attn_decode_noalloc", fn(_p(q), H, ctypes.byref(s), _p(kv_len), max_kv_len, _p(out), _p(lse), sc,
                                            num_splits, _p(err), _stream(stream)))
     return out
+
+
+def attn_prefill_chunk_workspace_size(B: int, T: int, G: int, d: int, layer_type: int, window: int) -> int:
+    fn = lib().olmo3_attn_prefill_chunk_workspace_size
+    fn.argtypes = [_i, _i, _i, _i, _i, _i]
+    fn.restype = ctypes.c_size_t
+    return int(fn(B, T, G, d, layer_type, window))
+
+
+def attn_prefill_chunk(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, cache: KVCache,
+                       pos_offset: torch.Tensor, scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                       lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                       err: Optional[torch.Tensor] = None, stream=None):
+    """A prompt chunk at positions pos_offset[b] + t attends over its cache and itself; the chunk
+    is appended to the cache.  Sliding layers need a workspace (allocated here if not given)."""
+    fn = lib().olmo3_attn_prefill_chunk
+    fn.argtypes = [_vp, _vp, _vp, ctypes.POINTER(CacheStruct), _vp, _i, _i, _vp, ctypes.c_float, _vp, _vp,
+                   ctypes.c_size_t, _vp, _vp]
+    fn.restype = _i
+    B, T, H, d = q.shape
+    _dev(q, "q", torch.bfloat16, (cache.B, T, H, cache.d))
+    _dev(k_new, "k_new", torch.bfloat16, (cache.B, T, cache.G, cache.d))
+    _dev(v_new, "v_new", torch.bfloat16, (cache.B, T, cache.G, cache.d))
+    _dev(pos_offset, "pos_offset", torch.int32, (cache.B,))
+    if out is None:
+        out = torch.empty_like(q)
+    _dev(out, "out", torch.bfloat16, (B, T, H, d))
+    if lse is not None:
+        _dev(lse, "lse", torch.float32, (B, H, T))
+    if err is not None:
+        _dev(err, "err", torch.int32)
+    need = attn_prefill_chunk_workspace_size(B, T, cache.G, d, cache.layer_type, cache.window)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    sc = 1.0 / math.sqrt(d) if scale is None else scale
+    s = cache.struct()
+    _check("olmo3_attn_prefill_chunk", fn(_p(q), _p(k_new), _p(v_new), ctypes.byref(s), _p(pos_offset), T, H,
+                                          _p(out), sc, _p(lse), _p(workspace), ws_bytes, _p(err), _stream(stream)))
+    return out

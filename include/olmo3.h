@@ -172,6 +172,34 @@ int olmo3_attn_prefill(const void *q, const void *k, const void *v, void *out,
                        float scale, float *lse_out, int *err_dev, void *stream);
 
 /*
+ * olmo3_attn_prefill_chunk - a chunk of T prompt tokens per sequence at positions
+ * pos_offset[b] + t attends over the cache of its sequence (the positions before
+ * the chunk) plus the chunk itself, and the chunk is appended to the cache.  This
+ * is prefill with a position offset into a live cache ([README] "Inference
+ * Pipeline": RoPE with position offsets for cache compatibility), so a long prompt
+ * can be fed in pieces; the result equals the rows of a one-shot prefill.
+ *   q           bf16 [B, T, H, d] after QK-norm + RoPE at positions pos_offset[b] + t.
+ *   k_new,v_new bf16 [B, T, G, d] (k_new after QK-norm + RoPE).
+ *   c           the layer's cache (HOST pointer to the struct), holding positions
+ *               0 .. pos_offset[b] - 1 of each sequence (the ring: its last window).
+ *   pos_offset  int32 [B].  out bf16 [B, T, H, d];  lse_out optional f32 [B, H, T].
+ *   Full layers: the chunk is appended first (it overwrites nothing), then the
+ *   chunk attends over cache rows 0 .. pos_offset + T - 1; no workspace is used.
+ *   Sliding layers: appending first would overwrite keys the chunk's early rows
+ *   still need, so the window [pos_offset - window + 1, pos_offset) is gathered from
+ *   the ring together with the chunk into `workspace`
+ *   (olmo3_attn_prefill_chunk_workspace_size bytes), attended, then the chunk is
+ *   appended.
+ *   Cache slots never written must hold finite values (allocate caches zeroed).
+ *   err_dev as for olmo3_kv_append and olmo3_attn_prefill.
+ */
+size_t olmo3_attn_prefill_chunk_workspace_size(int B, int T, int G, int d, int layer_type, int window);
+int olmo3_attn_prefill_chunk(const void *q, const void *k_new, const void *v_new,
+                             const olmo3_kv_cache *c, const int32_t *pos_offset, int T, int H,
+                             void *out, float scale, float *lse_out, void *workspace,
+                             size_t ws_bytes, int *err_dev, void *stream);
+
+/*
  * olmo3_attn_decode_workspace_size - bytes of f32 workspace olmo3_attn_decode
  * needs for these sizes (the split-KV partials).  max_kv_len is the largest
  * kv_len of the call; num_splits as for olmo3_attn_decode (0 = automatic).

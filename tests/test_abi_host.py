@@ -147,6 +147,24 @@ def test_decode_workspace_and_validation(lib):
         L.ERR_INVALID_ARG
 
 
+def test_prefill_chunk_workspace_and_validation(lib):
+    ws = L.attn_prefill_chunk_workspace_size
+    assert ws(2, 100, 8, 128, L.FULL, 4096) == 0                      # full layers read the cache in place
+    assert ws(2, 100, 8, 128, L.SLIDING, 4096) == 2 * 2 * (4095 + 100) * 8 * 128 * 2
+    assert ws(2, 100, 8, 96, L.SLIDING, 4096) == 0                    # unsupported d
+    f = lib.olmo3_attn_prefill_chunk
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(L.CacheStruct), ctypes.c_void_p,
+                  ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
+                  ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p]
+    c = _cache()  # sliding, window 16
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(c), FAKE, 8, 4, FAKE, 0.1, NULL, NULL, 0, NULL, NULL) == L.ERR_WORKSPACE
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(c), FAKE, 8, 3, FAKE, 0.1, NULL, FAKE, 1 << 20, NULL, NULL) == \
+        L.ERR_UNSUPPORTED                                               # H % G
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(c), NULL, 8, 4, FAKE, 0.1, NULL, FAKE, 1 << 20, NULL, NULL) == \
+        L.ERR_INVALID_ARG                                               # no pos_offset
+    assert f(FAKE, FAKE, FAKE, ctypes.byref(c), FAKE, 0, 4, FAKE, 0.1, NULL, NULL, 0, NULL, NULL) == L.OK
+
+
 def test_mask_and_layer_types_reject_bad_arguments(lib):
     assert lib.olmo3_layer_types(-1, None) == L.ERR_INVALID_ARG
     assert lib.olmo3_layer_types(3, None) == L.ERR_INVALID_ARG

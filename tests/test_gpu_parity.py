@@ -352,6 +352,79 @@ def test_decode_ragged_7b_full_size_sampled():
 
 
 # ---------------------------------------------------------------------------
+# Chunked prefill: a prompt chunk at an offset over a live cache
+# ---------------------------------------------------------------------------
+def _cache_from_oracle(ocs, typ, B, G, d, W, cap):
+    ck = torch.zeros((B * cap, G, d), dtype=torch.bfloat16, device="cuda")
+    cv = torch.zeros_like(ck)
+    for b, oc in enumerate(ocs):
+        valid = torch.from_numpy(oc.valid()).cuda()
+        ck[b * cap:(b + 1) * cap][valid] = bf16(oc.k[oc.valid()])
+        cv[b * cap:(b + 1) * cap][valid] = bf16(oc.v[oc.valid()])
+    return L.KVCache(typ, B, G, d, W, capacity=cap, k=ck, v=cv)
+
+
+@pytest.mark.parametrize("typ,W,H,G,d,p0s,T", [
+    (L.SLIDING, 256, 4, 2, 128, [0, 1, 255], 100),
+    (L.SLIDING, 256, 4, 2, 128, [256, 257, 600], 300),
+    (L.SLIDING, 128, 10, 2, 128, [130, 5], 1),
+    (L.SLIDING, 64, 2, 1, 64, [63, 64, 65], 77),
+    (L.FULL, 4096, 4, 4, 128, [0, 5, 700], 129),
+    (L.FULL, 4096, 10, 2, 128, [1000, 1], 300),
+    (L.FULL, 4096, 2, 1, 64, [64, 3], 1),
+])
+def test_prefill_chunk_parity(typ, W, H, G, d, p0s, T):
+    rng = np.random.default_rng(500 + T + sum(p0s))
+    B = len(p0s)
+    cap = W if typ == L.SLIDING else max(p0s) + T + 130
+    ocs = []
+    for p0 in p0s:
+        oc = O.KVCache(TYP[typ], cap, G, d)
+        first = max(0, p0 - cap) if typ == L.SLIDING else 0
+        if p0 > first:
+            oc.append(range(first, p0), f64(bf16(rng.standard_normal((p0 - first, G, d)), "cpu")),
+                      f64(bf16(rng.standard_normal((p0 - first, G, d)), "cpu")))
+        ocs.append(oc)
+    cache = _cache_from_oracle(ocs, typ, B, G, d, W, cap)
+    tq = bf16(rng.standard_normal((B, T, H, d)))
+    tk, tv = bf16(rng.standard_normal((B, T, G, d))), bf16(rng.standard_normal((B, T, G, d)))
+    lse = torch.empty((B, H, T), dtype=torch.float32, device="cuda")
+    err = new_err()
+    out = L.attn_prefill_chunk(tq, tk, tv, cache, torch.tensor(p0s, dtype=torch.int32, device="cuda"),
+                               lse=lse, err=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    ro, rl = O.chunk_attention(f64(tq), f64(tk), f64(tv), ocs, p0s, TYP[typ], W)
+    close_attn(f64(out), ro, "chunk out")
+    assert np.abs(lse.cpu().numpy() - rl).max() <= LSE_ABS
+    # the cache now holds the chunk too, exactly as the oracle's replay
+    kh, vh = f64(tk), f64(tv)
+    for b, oc in enumerate(ocs):
+        oc.append(range(p0s[b], p0s[b] + T), kh[b], vh[b])
+        got_k = f64(cache.k[b * cap:(b + 1) * cap])
+        np.testing.assert_array_equal(got_k[oc.valid()], oc.k[oc.valid()])
+
+
+@pytest.mark.parametrize("typ", [L.SLIDING, L.FULL])
+def test_chunked_prefill_equals_one_shot(typ):
+    rng = np.random.default_rng(77)
+    B, H, G, d, W, Ttot = 2, 4, 2, 128, 256, 1000
+    q, k, v = (rng.standard_normal((B, Ttot, n, d)) for n in (H, G, G))
+    tq, tk, tv = bf16(q), bf16(k), bf16(v)
+    ro, _ = O.prefill_attention(f64(tq), f64(tk), f64(tv), TYP[typ], W)
+    cache = L.KVCache(typ, B, G, d, W, capacity=Ttot + 64)
+    p0 = 0
+    for T in (300, 1, 255, 444):
+        pos = torch.full((B,), p0, dtype=torch.int32, device="cuda")
+        out = L.attn_prefill_chunk(tq[:, p0:p0 + T].contiguous(), tk[:, p0:p0 + T].contiguous(),
+                                   tv[:, p0:p0 + T].contiguous(), cache, pos)
+        torch.cuda.synchronize()
+        close_attn(f64(out), ro[:, p0:p0 + T], f"chunk at {p0}")
+        p0 += T
+    assert p0 == Ttot
+
+
+# ---------------------------------------------------------------------------
 # The toy configuration end to end: 6 layers, prefill 16 tokens, 8 decode steps
 # ---------------------------------------------------------------------------
 def test_toy_pipeline_full_parity():
