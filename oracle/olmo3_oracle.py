@@ -49,6 +49,7 @@ __all__ = [
     "attention_masks", "allowed", "allowed_count", "rms_norm", "rope_inv_freq",
     "rope", "qk_norm_rope", "attend", "prefill_attention", "KVCache",
     "append_slots", "decode_attention", "full_recompute_last_row", "chunk_attention",
+    "yarn_inv_freq", "yarn_mscale", "rope_with", "qk_norm_rope_with",
     "kv_bytes_per_token", "kv_cache_bytes",
 ]
 
@@ -137,6 +138,56 @@ def rope(x, positions, theta: float) -> np.ndarray:
     c, s = np.cos(ang), np.sin(ang)
     x1, x2 = x[..., :half], x[..., half:]
     return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+def yarn_inv_freq(d: int, theta: float, factor: float, original_context: int,
+                  beta_fast: float = 32.0, beta_slow: float = 1.0) -> np.ndarray:
+    """YaRN frequencies (Peng et al., 2023, "NTK-by-parts" interpolation).
+
+    [CASE] ingredient 7 and [SERVING]: RoPE of the full-attention layers is
+    rescaled with YaRN, factor 8 from the 8,192 positions of training.  The pages
+    give only the factor and the base context; the ramp bounds are the method's
+    (beta_fast = 32, beta_slow = 1): parity unpinned beyond factor 1 == plain RoPE.
+
+    Pair i turns r_i = original_context * theta^(-2i/d) / (2 pi) times over the
+    original context.  Pairs with r_i >= beta_fast keep their frequency, pairs with
+    r_i <= beta_slow are interpolated (frequency / factor), and a linear ramp in r_i
+    blends the two in between.
+    """
+    base = rope_inv_freq(d, theta)
+    if factor == 1.0:
+        return base
+    r = original_context * base / (2.0 * math.pi)
+    ramp = np.clip((r - beta_slow) / (beta_fast - beta_slow), 0.0, 1.0)  # 1 = keep, 0 = interpolate
+    return base * ramp + (base / factor) * (1.0 - ramp)
+
+
+def yarn_mscale(factor: float) -> float:
+    """YaRN attention temperature: q and k are both scaled by 0.1 ln(factor) + 1
+    (so the logits by its square); 1 for factor <= 1."""
+    return 1.0 if factor <= 1.0 else 0.1 * math.log(factor) + 1.0
+
+
+def rope_with(x, positions, inv_freq, out_scale: float = 1.0) -> np.ndarray:
+    """Rotate-half RoPE with an explicit frequency per pair, then a scale."""
+    x = np.asarray(x, dtype=np.float64)
+    half = x.shape[-1] // 2
+    ang = np.asarray(positions, dtype=np.float64)[..., None, None] * np.asarray(inv_freq, dtype=np.float64)
+    c, s = np.cos(ang), np.sin(ang)
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1) * out_scale
+
+
+def qk_norm_rope_with(q, k, gain_q, gain_k, positions, inv_freq, out_scale: float = 1.0,
+                      eps: float = 1e-6):
+    """QK-norm over the whole vector, then RoPE with the given frequencies and scale."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    B, T, H, d = q.shape
+    G = k.shape[2]
+    qn = rms_norm(q.reshape(B, T, H * d), gain_q, eps).reshape(B, T, H, d)
+    kn = rms_norm(k.reshape(B, T, G * d), gain_k, eps).reshape(B, T, G, d)
+    return rope_with(qn, positions, inv_freq, out_scale), rope_with(kn, positions, inv_freq, out_scale)
 
 
 def qk_norm_rope(q, k, gain_q, gain_k, positions, eps: float = 1e-6,

@@ -361,6 +361,28 @@ def test_chunked_prefill_equals_one_shot_prefill(typ):
     assert p0 == Ttot
 
 
+def test_yarn_factor_one_is_plain_rope():
+    # the only pin the pages allow: YaRN with factor 1 is plain RoPE (no interpolation, no temperature)
+    rng = np.random.default_rng(13)
+    x = rng.standard_normal((3, 2, 128))
+    pos = np.array([0, 77, 65535])
+    np.testing.assert_array_equal(O.yarn_inv_freq(128, 5e5, 1.0, 8192), O.rope_inv_freq(128, 5e5))
+    assert O.yarn_mscale(1.0) == 1.0
+    np.testing.assert_allclose(O.rope_with(x, pos, O.yarn_inv_freq(128, 5e5, 1.0, 8192), O.yarn_mscale(1.0)),
+                               O.rope(x, pos, 5e5), atol=1e-12)
+
+
+def test_yarn_limits_of_the_ramp():
+    # the definition's two ends: fast pairs keep their frequency, slow pairs are divided by the factor
+    base = O.rope_inv_freq(128, 5e5)
+    f = O.yarn_inv_freq(128, 5e5, 8.0, 8192)
+    r = 8192 * base / (2 * math.pi)
+    np.testing.assert_allclose(f[r >= 32], base[r >= 32], rtol=1e-15)
+    np.testing.assert_allclose(f[r <= 1], base[r <= 1] / 8, rtol=1e-15)
+    assert np.all(f <= base) and np.all(f >= base / 8)
+    assert abs(O.yarn_mscale(8.0) - (1 + 0.1 * math.log(8))) < 1e-15
+
+
 def test_kv_sizing_matches_the_pages():
     g = {r[0]: float(r[1]) for r in read_golden("kv_sizing.txt")}
     t32 = O.layer_types(32)
