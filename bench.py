@@ -48,7 +48,9 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="7b-prefill",
-                    choices=["7b-prefill", "32b-prefill", "7b-decode", "32b-decode", "ragged-7b-decode"])
+                    choices=["7b-prefill", "32b-prefill", "7b-decode", "32b-decode", "ragged-7b-decode",
+                             "7b-prefill-chunked", "32b-prefill-chunked"])
+    ap.add_argument("--chunk", type=int, default=2048, help="prompt chunk of the *-prefill-chunked workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -154,9 +156,11 @@ class ClockSampler:
 # --------------------------------------------------------------------------
 class PrefillStep:
     """Prefill of T tokens on one sliding and one full layer, then one decode
-    token per layer, through the C ABI."""
+    token per layer, through the C ABI.  With chunk > 0 the prompt goes in
+    pieces of `chunk` tokens through the chunked-prefill entry point (each piece
+    attends over the cache the earlier pieces filled)."""
 
-    def __init__(self, name, dev, stream):
+    def __init__(self, name, dev, stream, chunk=0):
         from hybrid_sliding_window_olmo3_b200 import olmo3 as L
         from hybrid_sliding_window_olmo3_b200 import workloads as WL
         self.L = L
@@ -164,7 +168,7 @@ class PrefillStep:
         sh = wl.shape
         self.wl, self.sh, self.dev, self.stream = wl, sh, dev, stream
         B, T, H, G, d, W = wl.B, wl.T, sh.H, sh.G, sh.d, sh.window
-        self.B, self.T = B, T
+        self.B, self.T, self.chunk = B, T, chunk
         types = L.layer_types(sh.n_layers)
         self.layers = []
         for li in wl.layers:
@@ -186,20 +190,39 @@ class PrefillStep:
             lay["out1"] = torch.empty(B, H, d, dtype=torch.bfloat16, device=dev)
             n_ws = L.attn_decode_workspace_size(B, H, G, d, T + 1, typ, W)
             lay["ws"] = torch.empty(max(n_ws // 4, 4), dtype=torch.float32, device=dev)
+            if chunk:
+                n_cw = L.attn_prefill_chunk_workspace_size(B, chunk, G, d, typ, W)
+                lay["cws"] = torch.empty(max(n_cw, 16), dtype=torch.uint8, device=dev)
+                lay["chunks"] = []
+                for c0 in range(0, T, chunk):
+                    c1 = min(T, c0 + chunk)
+                    lay["chunks"].append(dict(
+                        c0=c0, q=lay["q"][:, c0:c1].contiguous(), k=lay["k"][:, c0:c1].contiguous(),
+                        v=lay["v"][:, c0:c1].contiguous(),
+                        qh=torch.empty(B, c1 - c0, H, d, dtype=torch.bfloat16, device=dev),
+                        kh=torch.empty(B, c1 - c0, G, d, dtype=torch.bfloat16, device=dev),
+                        out=torch.empty(B, c1 - c0, H, d, dtype=torch.bfloat16, device=dev),
+                        pos=torch.full((B,), c0, dtype=torch.int32, device=dev)))
             lay["flops"] = prefill_flops(B, T, H, d, W, typ == L.FULL)
             self.layers.append(lay)
         self.pos0 = torch.zeros(B, dtype=torch.int32, device=dev)
         self.posT = torch.full((B,), T, dtype=torch.int32, device=dev)
         self.kvlen = torch.full((B,), T + 1, dtype=torch.int32, device=dev)
         self.flops_per_step = sum(x["flops"] for x in self.layers)
-        self.launches_per_step = 7 * len(self.layers)
+        n_chunks = len(self.layers[0].get("chunks", [])) if chunk else 0
+        # one-shot: qknorm, append, prefill, qknorm, append, decode + combine per layer;
+        # chunked: per chunk qknorm + chunk call (gather, prefill, append on sliding layers;
+        # append, prefill on full layers), then the decode token
+        self.launches_per_step = (7 * len(self.layers) if not chunk else
+                                  sum(n_chunks * (1 + (3 if x["typ"] == L.SLIDING else 2)) + 4 for x in self.layers))
         self.unit = "TFLOP/s"
         self.h2d = sum(t.numel() * t.element_size() for lay in self.layers for n, t in lay["host"].items())
         self.d2h = sum(lay["out"].numel() * 2 + lay["out1"].numel() * 2 for lay in self.layers)
         self.config = {
             "workload": f"OLMo 3 {sh.name[6:]} prefill attention: B={B}, T={T}, H={H}, G={G}, d={d}, window {W}, "
                         f"layers {list(wl.layers)} (types {[x['typ'] for x in self.layers]}, 0=sliding 1=full), "
-                        "then one decode token per layer",
+                        + (f"prompt in chunks of {chunk} tokens through the chunked-prefill call, " if chunk else "")
+                        + "then one decode token per layer",
             "global_batch": B, "seq_len": T,
             "l2": f"inputs larger than L2 ({self.h2d / 2**20:.0f} MiB read per step)",
             "parallelism": "replicas",
@@ -213,16 +236,29 @@ class PrefillStep:
             if host_io:
                 for n in ("q", "k", "v", "gq", "gk", "q1", "k1", "v1"):
                     lay[n].copy_(lay["host"][n], non_blocking=True)
-            L.qknorm_rope(lay["q"], lay["k"], lay["gq"], lay["gk"], self.pos0, q_out=lay["qh"], k_out=lay["kh"],
-                          stream=s)
-            L.kv_append(lay["cache"], lay["kh"], lay["v"], self.pos0, stream=s)
-            if timed_kernel:
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(s)
-            L.attn_prefill(lay["qh"], lay["kh"], lay["v"], lay["typ"], self.sh.window, out=lay["out"], stream=s)
-            if timed_kernel:
-                e1.record(s)
-                self.ev.append((e0, e1, lay["flops"]))
+            if self.chunk:
+                if timed_kernel:
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(s)
+                for ch in lay["chunks"]:
+                    L.qknorm_rope(ch["q"], ch["k"], lay["gq"], lay["gk"], ch["pos"], q_out=ch["qh"], k_out=ch["kh"],
+                                  stream=s)
+                    L.attn_prefill_chunk(ch["qh"], ch["kh"], ch["v"], lay["cache"], ch["pos"], out=ch["out"],
+                                         workspace=lay["cws"], stream=s)
+                if timed_kernel:
+                    e1.record(s)
+                    self.ev.append((e0, e1, lay["flops"]))
+            else:
+                L.qknorm_rope(lay["q"], lay["k"], lay["gq"], lay["gk"], self.pos0, q_out=lay["qh"],
+                              k_out=lay["kh"], stream=s)
+                L.kv_append(lay["cache"], lay["kh"], lay["v"], self.pos0, stream=s)
+                if timed_kernel:
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(s)
+                L.attn_prefill(lay["qh"], lay["kh"], lay["v"], lay["typ"], self.sh.window, out=lay["out"], stream=s)
+                if timed_kernel:
+                    e1.record(s)
+                    self.ev.append((e0, e1, lay["flops"]))
             L.qknorm_rope(lay["q1"], lay["k1"], lay["gq"], lay["gk"], self.posT, q_out=lay["qh1"],
                           k_out=lay["kh1"], stream=s)
             L.kv_append(lay["cache"], lay["kh1"], lay["v1"], self.posT, stream=s)
@@ -245,7 +281,8 @@ class PrefillStep:
         return {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4), "peak_kind": "measured burst cuBLAS bf16"
                 if peaks is not FALLBACK_PEAKS else "fallback burst",
-                "kernel": self.kernel_name, "launches": len(self.ev),
+                "kernel": self.kernel_name if not self.chunk else
+                "qknorm_rope + attn_prefill_chunk over all chunks of a layer", "launches": len(self.ev),
                 "avg_launch_ms": round(tot_ms / max(len(self.ev), 1), 4)}
 
     def cpu_baseline(self, seconds, rows_per_block=16):
@@ -479,9 +516,11 @@ class DecodeStep:
                           f"one sliding and one full layer), {el:.1f} s of oracle time; numpy, single thread"}
 
 
-def make_workload(name, dev, stream, batch=0, shared=False):
+def make_workload(name, dev, stream, batch=0, shared=False, chunk=0):
     if name.endswith("prefill"):
         return PrefillStep(name, dev, stream)
+    if name.endswith("prefill-chunked"):
+        return PrefillStep(name[:-len("-chunked")], dev, stream, chunk=chunk)
     return DecodeStep(name, dev, stream, batch, shared)
 
 
@@ -497,7 +536,7 @@ def run_ours(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
     stream = torch.cuda.current_stream(dev)
-    wk = make_workload(args.workload, dev, stream, args.batch, args.shared_caches)
+    wk = make_workload(args.workload, dev, stream, args.batch, args.shared_caches, args.chunk)
     peaks, peak_src = load_peaks()
 
     def barrier():
@@ -586,7 +625,8 @@ def run_reference(args):
     if dev is None:
         print(json.dumps({"impl": "reference", "unavailable": "the sampled workload is generated on a CUDA device"}))
         return
-    wk = make_workload(args.workload, dev, torch.cuda.current_stream(dev), args.batch, args.shared_caches)
+    wk = make_workload(args.workload, dev, torch.cuda.current_stream(dev), args.batch, args.shared_caches,
+                       args.chunk)
     per = []
     for i in range(args.warmup + args.steps):
         cb = wk.cpu_baseline(max(2.0, min(8.0, 150.0 / (args.warmup + args.steps))))

@@ -11,7 +11,8 @@
 namespace olmo3 {
 
 struct RopeTable {
-  double inv_freq[64];  // theta^(-2i/d), i < d/2
+  double inv_freq[64];  // angle per position of pair i < d/2 (theta^(-2i/d) for plain RoPE)
+  float out_scale;      // applied to the rotated q and k (1; YaRN's attention temperature)
 };
 
 cudaError_t launch_qknorm_rope(const void *q, const void *k, const void *v, int in_dtype, const float *gain_q,

@@ -102,11 +102,11 @@ int olmo3_attn_mask(int T, int window, int layer_type, uint8_t *out_dev, void *s
   return cuda_status(launch_attn_mask(T, window, layer_type, out_dev, as_stream(stream)));
 }
 
-int olmo3_qknorm_rope(const void *q, const void *k, const void *v, int in_dtype, const float *gain_q,
-                      const float *gain_k, void *q_out, void *k_out, void *v_out, const int32_t *pos_offset, int B,
-                      int T, int H, int G, int d, float eps, double theta, void *stream) {
-  if (B < 0 || T < 0 || H < 1 || G < 1 || !(eps >= 0.f) || !(theta > 0.0) ||
-      (in_dtype != OLMO3_F32 && in_dtype != OLMO3_BF16))
+namespace {
+int qknorm_rope_common(const void *q, const void *k, const void *v, int in_dtype, const float *gain_q,
+                       const float *gain_k, void *q_out, void *k_out, void *v_out, const int32_t *pos_offset, int B,
+                       int T, int H, int G, int d, float eps, const RopeTable &tab, void *stream) {
+  if (B < 0 || T < 0 || H < 1 || G < 1 || !(eps >= 0.f) || (in_dtype != OLMO3_F32 && in_dtype != OLMO3_BF16))
     return OLMO3_ERR_INVALID_ARG;
   if (!valid_d(d)) return OLMO3_ERR_UNSUPPORTED;
   if (H * d > 8192 || G * d > 8192) return OLMO3_ERR_UNSUPPORTED;
@@ -118,10 +118,51 @@ int olmo3_qknorm_rope(const void *q, const void *k, const void *v, int in_dtype,
   for (const void *p : ptrs)
     if (!aligned16(p)) return OLMO3_ERR_INVALID_ARG;
   if (v_out && (!aligned16(v) || !aligned16(v_out))) return OLMO3_ERR_INVALID_ARG;
-  RopeTable tab;
-  for (int i = 0; i < 64; ++i) tab.inv_freq[i] = i < d / 2 ? pow(theta, -2.0 * i / d) : 0.0;
   return cuda_status(launch_qknorm_rope(q, k, v, in_dtype, gain_q, gain_k, q_out, k_out, v_out, pos_offset, B, T,
                                         H, G, d, eps, tab, as_stream(stream)));
+}
+}  // namespace
+
+int olmo3_qknorm_rope(const void *q, const void *k, const void *v, int in_dtype, const float *gain_q,
+                      const float *gain_k, void *q_out, void *k_out, void *v_out, const int32_t *pos_offset, int B,
+                      int T, int H, int G, int d, float eps, double theta, void *stream) {
+  if (!(theta > 0.0)) return OLMO3_ERR_INVALID_ARG;
+  RopeTable tab;
+  for (int i = 0; i < 64; ++i) tab.inv_freq[i] = i < d / 2 ? pow(theta, -2.0 * i / d) : 0.0;
+  tab.out_scale = 1.0f;
+  return qknorm_rope_common(q, k, v, in_dtype, gain_q, gain_k, q_out, k_out, v_out, pos_offset, B, T, H, G, d, eps,
+                            tab, stream);
+}
+
+int olmo3_qknorm_rope_yarn(const void *q, const void *k, const void *v, int in_dtype, const float *gain_q,
+                           const float *gain_k, void *q_out, void *k_out, void *v_out, const int32_t *pos_offset,
+                           int B, int T, int H, int G, int d, float eps, double theta, double factor,
+                           int original_context, double beta_fast, double beta_slow, void *stream) {
+  if (!(theta > 0.0) || !(factor >= 1.0) || original_context < 1 || !(beta_fast > beta_slow))
+    return OLMO3_ERR_INVALID_ARG;
+  // NTK-by-parts: pair i turns r = original_context * f_i / (2 pi) times over the
+  // original context; it keeps f_i when r >= beta_fast, becomes f_i / factor when
+  // r <= beta_slow, and blends linearly in between.
+  RopeTable tab;
+  const double two_pi = 6.283185307179586476925286766559;
+  for (int i = 0; i < 64; ++i) {
+    if (i >= d / 2) {
+      tab.inv_freq[i] = 0.0;
+      continue;
+    }
+    const double f = pow(theta, -2.0 * i / d);
+    if (factor == 1.0) {
+      tab.inv_freq[i] = f;
+      continue;
+    }
+    const double r = original_context * f / two_pi;
+    double keep = (r - beta_slow) / (beta_fast - beta_slow);
+    keep = keep < 0.0 ? 0.0 : (keep > 1.0 ? 1.0 : keep);
+    tab.inv_freq[i] = f * keep + (f / factor) * (1.0 - keep);
+  }
+  tab.out_scale = factor > 1.0 ? static_cast<float>(0.1 * log(factor) + 1.0) : 1.0f;
+  return qknorm_rope_common(q, k, v, in_dtype, gain_q, gain_k, q_out, k_out, v_out, pos_offset, B, T, H, G, d, eps,
+                            tab, stream);
 }
 
 int olmo3_kv_append(const olmo3_kv_cache *c, const void *k_new, const void *v_new, const int32_t *pos_offset,

@@ -124,8 +124,8 @@ __global__ void __launch_bounds__(kNormThreads) qknorm_rope_kernel(
     const double p = static_cast<double>(pos_offset[b]) + static_cast<double>(t);
     double sn, cs;
     sincos(p * tab.inv_freq[threadIdx.x], &sn, &cs);
-    s_cos[threadIdx.x] = static_cast<float>(cs);
-    s_sin[threadIdx.x] = static_cast<float>(sn);
+    s_cos[threadIdx.x] = static_cast<float>(cs) * tab.out_scale;
+    s_sin[threadIdx.x] = static_cast<float>(sn) * tab.out_scale;
   }
   const float tq = block_sum(ssq_q, s_red[0]);
   const float tk = block_sum(ssq_k, s_red[1]);  // its __syncthreads also publishes s_cos / s_sin

@@ -320,3 +320,36 @@ def attn_prefill_chunk(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor
     _check("olmo3_attn_prefill_chunk", fn(_p(q), _p(k_new), _p(v_new), ctypes.byref(s), _p(pos_offset), T, H,
                                           _p(out), sc, _p(lse), _p(workspace), ws_bytes, _p(err), _stream(stream)))
     return out
+
+
+def qknorm_rope_yarn(q: torch.Tensor, k: torch.Tensor, gain_q: torch.Tensor, gain_k: torch.Tensor,
+                     pos_offset: torch.Tensor, eps: float = 1e-6, theta: float = 500000.0, factor: float = 8.0,
+                     original_context: int = 8192, beta_fast: float = 32.0, beta_slow: float = 1.0,
+                     v: Optional[torch.Tensor] = None, q_out=None, k_out=None, v_out=None, stream=None):
+    """qknorm_rope with YaRN-rescaled RoPE (for the full-attention layers of the long-context model)."""
+    fn = lib().olmo3_qknorm_rope_yarn
+    fn.argtypes = [_vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float,
+                   ctypes.c_double, ctypes.c_double, _i, ctypes.c_double, ctypes.c_double, _vp]
+    fn.restype = _i
+    B, T, H, d = q.shape
+    G = k.shape[2]
+    if q.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("q must be float32 or bfloat16")
+    in_dtype = F32 if q.dtype == torch.float32 else BF16
+    _dev(q, "q")
+    _dev(k, "k", q.dtype, (B, T, G, d))
+    _dev(gain_q, "gain_q", torch.float32, (H * d,))
+    _dev(gain_k, "gain_k", torch.float32, (G * d,))
+    _dev(pos_offset, "pos_offset", torch.int32, (B,))
+    q_out = torch.empty((B, T, H, d), dtype=torch.bfloat16, device=q.device) if q_out is None else q_out
+    k_out = torch.empty((B, T, G, d), dtype=torch.bfloat16, device=q.device) if k_out is None else k_out
+    _dev(q_out, "q_out", torch.bfloat16, (B, T, H, d))
+    _dev(k_out, "k_out", torch.bfloat16, (B, T, G, d))
+    if v is not None:
+        _dev(v, "v", q.dtype, (B, T, G, d))
+        v_out = torch.empty((B, T, G, d), dtype=torch.bfloat16, device=q.device) if v_out is None else v_out
+        _dev(v_out, "v_out", torch.bfloat16, (B, T, G, d))
+    _check("olmo3_qknorm_rope_yarn", fn(_p(q), _p(k), _p(v), in_dtype, _p(gain_q), _p(gain_k), _p(q_out), _p(k_out),
+                                        _p(v_out), _p(pos_offset), B, T, H, G, d, eps, theta, factor,
+                                        original_context, beta_fast, beta_slow, _stream(stream)))
+    return q_out, k_out, v_out

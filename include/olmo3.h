@@ -110,6 +110,26 @@ int olmo3_qknorm_rope(const void *q, const void *k, const void *v, int in_dtype,
                       float eps, double theta, void *stream);
 
 /*
+ * olmo3_qknorm_rope_yarn - olmo3_qknorm_rope with YaRN-rescaled RoPE, for the
+ * full-attention layers of the long-context model ([CASE] ingredient 7: RoPE on the
+ * full layers is rescaled with YaRN from the 8,192 training positions to 65,536;
+ * [SERVING]: factor 8 from an 8192 base).  The pages give only the factor and the
+ * base; the rest is the YaRN method's "NTK-by-parts" rule: pair i turns
+ * r = original_context * f_i / (2 pi) times over the original context, keeps its
+ * frequency f_i = theta^(-2i/d) when r >= beta_fast, uses f_i / factor when
+ * r <= beta_slow, and blends linearly in between; the rotated q and k are both
+ * multiplied by 0.1 ln(factor) + 1 (the attention temperature).  factor == 1 is
+ * exactly olmo3_qknorm_rope.  Typical: factor 8, original_context 8192,
+ * beta_fast 32, beta_slow 1.  Other arguments as olmo3_qknorm_rope.
+ */
+int olmo3_qknorm_rope_yarn(const void *q, const void *k, const void *v, int in_dtype,
+                           const float *gain_q, const float *gain_k,
+                           void *q_out, void *k_out, void *v_out,
+                           const int32_t *pos_offset, int B, int T, int H, int G, int d,
+                           float eps, double theta, double factor, int original_context,
+                           double beta_fast, double beta_slow, void *stream);
+
+/*
  * olmo3_kv_cache - a preallocated per-layer-type cache ([SERVING]: per-layer-type
  * cache management; replaces the concatenation-grown cache of [README] "KV Cache
  * Implementation").

@@ -49,7 +49,7 @@ __all__ = [
     "attention_masks", "allowed", "allowed_count", "rms_norm", "rope_inv_freq",
     "rope", "qk_norm_rope", "attend", "prefill_attention", "KVCache",
     "append_slots", "decode_attention", "full_recompute_last_row", "chunk_attention",
-    "yarn_inv_freq", "yarn_mscale", "rope_with", "qk_norm_rope_with",
+    "yarn_inv_freq", "yarn_mscale", "rope_with", "qk_norm_rope_with", "out_proj_postnorm_residual",
     "kv_bytes_per_token", "kv_cache_bytes",
 ]
 
@@ -258,6 +258,19 @@ def prefill_attention(q, k, v, layer_type: str, window: int,
         rows = np.arange(T)
     rows = np.asarray(rows)
     return attend(q[:, rows], pos[:, rows], k, pos, v, layer_type, window, scale)
+
+
+def out_proj_postnorm_residual(x, attn, w_o, gain, eps: float = 1e-6):
+    """[CASE] ingredients 1 and 6: the bias-free output projection, then the
+    reordered norm h = x + RMSNorm(attn W_o^T) with one gain per model feature.
+
+    x: [M, D] residual stream; attn: [M, H*d] attention output (heads side by
+    side); w_o: [D, H*d] (row j maps the attention features to model feature j);
+    gain: [D].  Returns h [M, D] in float64.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    y = np.asarray(attn, dtype=np.float64) @ np.asarray(w_o, dtype=np.float64).T
+    return x + rms_norm(y, gain, eps)
 
 
 # ---------------------------------------------------------------------------

@@ -109,6 +109,25 @@ def test_qknorm_rope_parity(B, T, H, G, d, dt, offs):
     assert torch.equal(vo.cpu(), tv.cpu().to(torch.bfloat16))
 
 
+@pytest.mark.parametrize("factor,offs", [(8.0, [0, 8191, 65535]), (4.0, [100, 30000, 7]), (1.0, [5, 60000, 1])])
+def test_qknorm_rope_yarn_parity(factor, offs):
+    rng = np.random.default_rng(150)
+    B, T, H, G, d = 3, 4, 32, 32, 128
+    tq, tk = bf16(rng.standard_normal((B, T, H, d)) * 2), bf16(rng.standard_normal((B, T, G, d)) * 2)
+    gq = torch.rand(H * d, device="cuda") + 0.5
+    gk = torch.rand(G * d, device="cuda") + 0.5
+    pos = torch.tensor(offs, dtype=torch.int32, device="cuda")
+    qh, kh, _ = L.qknorm_rope_yarn(tq, tk, gq, gk, pos, factor=factor, original_context=8192)
+    inv = O.yarn_inv_freq(d, 5e5, factor, 8192, 32.0, 1.0)
+    positions = np.array(offs)[:, None] + np.arange(T)[None, :]
+    rq, rk = O.qk_norm_rope_with(f64(tq), f64(tk), f64(gq), f64(gk), positions, inv, O.yarn_mscale(factor))
+    close_qk(f64(qh), rq, "yarn q_hat")
+    close_qk(f64(kh), rk, "yarn k_hat")
+    if factor == 1.0:  # the same table as plain RoPE: bit for bit
+        pq, pk, _ = L.qknorm_rope(tq, tk, gq, gk, pos)
+        assert torch.equal(pq, qh) and torch.equal(pk, kh)
+
+
 def test_qknorm_rope_in_place():
     rng = np.random.default_rng(7)
     B, T, H, G, d = 2, 9, 8, 4, 128

@@ -383,6 +383,26 @@ def test_yarn_limits_of_the_ramp():
     assert abs(O.yarn_mscale(8.0) - (1 + 0.1 * math.log(8))) < 1e-15
 
 
+def test_reordered_norm_example():
+    g = {r[0]: [float(x) for x in r[1:]] for r in read_golden("reordered_norm_example.txt")}
+    attn = np.array([g["attention_output"]])
+    x = np.array([[0.25, -2.0]])
+    h = O.out_proj_postnorm_residual(x, attn, np.eye(2), np.ones(2))
+    np.testing.assert_allclose(h - x, [g["added"]], atol=0.005)   # the norm acts on the output, before the add
+    h3 = O.out_proj_postnorm_residual(x, attn, np.eye(2), np.array([3.0, 0.5]))
+    np.testing.assert_allclose(h3 - x, [[3 * 0.8485281, 0.5 * 1.1313708]], atol=1e-6)  # times the gain
+
+
+def test_out_projection_is_a_plain_matmul():
+    # with a gain of zero only the residual survives; with identity weights the projection is the identity
+    rng = np.random.default_rng(14)
+    x, a = rng.standard_normal((4, 6)), rng.standard_normal((4, 6))
+    np.testing.assert_array_equal(O.out_proj_postnorm_residual(x, a, rng.standard_normal((6, 6)), np.zeros(6)), x)
+    w = rng.standard_normal((6, 6))
+    ref = x + O.rms_norm(np.einsum("mk,nk->mn", a, w), np.ones(6))
+    np.testing.assert_allclose(O.out_proj_postnorm_residual(x, a, w, np.ones(6)), ref, atol=1e-12)
+
+
 def test_kv_sizing_matches_the_pages():
     g = {r[0]: float(r[1]) for r in read_golden("kv_sizing.txt")}
     t32 = O.layer_types(32)
