@@ -49,7 +49,7 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="7b-prefill",
                     choices=["7b-prefill", "32b-prefill", "7b-decode", "32b-decode", "ragged-7b-decode",
-                             "7b-prefill-chunked", "32b-prefill-chunked"])
+                             "7b-prefill-chunked", "32b-prefill-chunked", "7b-out-proj", "32b-out-proj"])
     ap.add_argument("--chunk", type=int, default=2048, help="prompt chunk of the *-prefill-chunked workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -516,7 +516,92 @@ class DecodeStep:
                           f"one sliding and one full layer), {el:.1f} s of oracle time; numpy, single thread"}
 
 
+class OutProjStep:
+    """The attention block's output side for a whole prompt: h = x + RMSNorm(attn W_o^T) * gain
+    (tcgen05 GEMM with row sums of squares, then the norm + residual finisher)."""
+
+    def __init__(self, name, dev, stream):
+        from hybrid_sliding_window_olmo3_b200 import olmo3 as L
+        from hybrid_sliding_window_olmo3_b200 import workloads as WL
+        self.L = L
+        wl = WL.WORKLOADS[name.replace("out-proj", "prefill")]
+        sh = wl.shape
+        self.sh, self.dev, self.stream = sh, dev, stream
+        M, K = wl.B * wl.T, sh.H * sh.d
+        D = {"olmo3-7b": 4096, "olmo3-32b": 5120}[sh.name]
+        self.M, self.D, self.K = M, D, K
+        host = dict(attn=WL.randn_bf16((M, K), wl.seed + 11), x=WL.randn_bf16((M, D), wl.seed + 12),
+                    w=(WL.randn_bf16((D, K), wl.seed + 13).float() / K ** 0.5).to(torch.bfloat16),
+                    g=torch.rand(D, generator=torch.Generator().manual_seed(wl.seed)) + 0.5)
+        self.host = {n: t.pin_memory() for n, t in host.items()}
+        for n, t in host.items():
+            setattr(self, n, t.to(dev))
+        self.h = torch.empty(M, D, dtype=torch.bfloat16, device=dev)
+        self.h_host = torch.empty(M, D, dtype=torch.bfloat16).pin_memory()
+        self.ws = torch.empty(L.out_proj_workspace_size(M, D), dtype=torch.uint8, device=dev)
+        self.flops = 2 * M * D * K
+        self.unit = "TFLOP/s"
+        self.launches_per_step = 2  # GEMM + finisher (plus a memset of the row sums)
+        self.h2d = sum(t.numel() * t.element_size() for t in self.host.values())
+        self.d2h = M * D * 2
+        self.ev = []
+        self.kernel_file, self.kernel_name = "out_proj.cu", "gemm_rowss_kernel + postnorm_residual_kernel"
+        self.config = {"workload": f"OLMo 3 {sh.name[6:]} attention output side: h = x + RMSNorm(attn W_o^T), "
+                                   f"M={M} tokens, K={K}, D={D}, bf16",
+                       "global_batch": wl.B, "seq_len": wl.T, "l2": "inputs larger than L2", "parallelism": "replicas"}
+
+    def step(self, timed_kernel=False, host_io=False):
+        s = self.stream
+        if host_io:
+            for n in ("attn", "x", "w", "g"):
+                getattr(self, n).copy_(self.host[n], non_blocking=True)
+        if timed_kernel:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+        self.L.out_proj_postnorm_residual(self.attn, self.w, self.g, self.x, h_out=self.h, workspace=self.ws,
+                                          stream=s)
+        if timed_kernel:
+            e1.record(s)
+            self.ev.append((e0, e1, self.flops))
+        if host_io:
+            self.h_host.copy_(self.h, non_blocking=True)
+
+    def work_per_step(self):
+        return self.flops / 1e12
+
+    def kernel_roofline(self, peaks):
+        tot_ms = sum(e0.elapsed_time(e1) for e0, e1, _ in self.ev)
+        achieved = sum(f for _, _, f in self.ev) / (tot_ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops"]
+        return {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "peak_kind": "measured burst cuBLAS bf16",
+                "kernel": self.kernel_name, "launches": len(self.ev),
+                "avg_launch_ms": round(tot_ms / max(len(self.ev), 1), 4)}
+
+    def cpu_baseline(self, seconds):
+        import oracle.olmo3_oracle as O
+        a, w, x, g = (self.host[n].float().numpy() for n in ("attn", "w", "x", "g"))
+        done, el, rows = 0, 0.0, 0
+        rng = np.random.default_rng(0)
+        while el < seconds:
+            r = rng.integers(0, self.M, 8)
+            t0 = time.perf_counter()
+            O.out_proj_postnorm_residual(x[r], a[r], w, g)
+            el += time.perf_counter() - t0
+            done += 2 * 8 * self.D * self.K
+            rows += 8
+        try:
+            from threadpoolctl import threadpool_info
+            cores = max([i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"] or [1])
+        except Exception:  # noqa: BLE001 - reporting only
+            cores = len(os.sched_getaffinity(0))
+        return {"value": done / el / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                "sample": f"{rows} rows (fp64 matmul with W_o, norm, residual), {el:.1f} s; numpy (BLAS threads)"}
+
+
 def make_workload(name, dev, stream, batch=0, shared=False, chunk=0):
+    if name.endswith("out-proj"):
+        return OutProjStep(name, dev, stream)
     if name.endswith("prefill"):
         return PrefillStep(name, dev, stream)
     if name.endswith("prefill-chunked"):

@@ -64,4 +64,9 @@ cudaError_t launch_gather_window(const olmo3_kv_cache &c, const void *k_new, con
                                  const int32_t *pos_offset, int T, int Tk, void *k_out, void *v_out,
                                  cudaStream_t stream);
 
+// Y = A B^T (tcgen05) with per-row sums of squares, then h = x + Y rsqrt(ss/N + eps) gain.
+// tmA: 2-d map over A [M, K] with 64 x 128 boxes; tmB: over B [N, K] with 64 x 256 boxes.
+cudaError_t launch_out_proj(const CUtensorMap &tmA, const CUtensorMap &tmB, void *Y, float *ss, const float *gain,
+                            const void *x, void *h, int M, int N, int K, float eps, int *err, cudaStream_t stream);
+
 }  // namespace olmo3

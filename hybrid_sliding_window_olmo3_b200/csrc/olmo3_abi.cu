@@ -243,6 +243,38 @@ int olmo3_attn_prefill_chunk(const void *q, const void *k_new, const void *v_new
   return cuda_status(launch_kv_append(*c, k_new, v_new, pos_offset, T, nullptr, err_dev, s));
 }
 
+size_t olmo3_out_proj_workspace_size(int M, int D) {
+  if (M < 0 || D < 1) return 0;
+  const size_t y = (static_cast<size_t>(M) * D * 2 + 255) & ~static_cast<size_t>(255);
+  return y + static_cast<size_t>(M) * 4;
+}
+
+int olmo3_out_proj_postnorm_residual(const void *attn, const void *w_o, const float *gain, const void *x, void *h_out,
+                                     int M, int D, int K, float eps, void *workspace, size_t ws_bytes, int *err_dev,
+                                     void *stream) {
+  if (M < 0 || D < 1 || K < 1 || !(eps >= 0.f)) return OLMO3_ERR_INVALID_ARG;
+  if (K % 64 != 0 || D % 8 != 0 || M > 65535 * 128 || static_cast<int64_t>(M) * D >= (int64_t(1) << 31))
+    return OLMO3_ERR_UNSUPPORTED;
+  if (M == 0) return OLMO3_OK;
+  if (!attn || !w_o || !gain || !x || !h_out) return OLMO3_ERR_INVALID_ARG;
+  const void *ptrs[] = {attn, w_o, gain, x, h_out};
+  for (const void *p : ptrs)
+    if (!aligned16(p)) return OLMO3_ERR_INVALID_ARG;
+  const size_t need = olmo3_out_proj_workspace_size(M, D);
+  if (workspace == nullptr || ws_bytes < need || !aligned16(workspace)) return OLMO3_ERR_WORKSPACE;
+  CUtensorMap tmA, tmB;
+  const cuuint32_t box_a[2] = {64, 128}, box_b[2] = {64, 256};
+  const cuuint64_t dims_a[2] = {(cuuint64_t)K, (cuuint64_t)M}, dims_b[2] = {(cuuint64_t)K, (cuuint64_t)D};
+  const cuuint64_t stride[1] = {(cuuint64_t)K * 2};
+  if (!encode_bf16(&tmA, attn, 2, dims_a, stride, box_a, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_bf16(&tmB, w_o, 2, dims_b, stride, box_b, CU_TENSOR_MAP_SWIZZLE_128B))
+    return OLMO3_ERR_CUDA;
+  void *Y = workspace;
+  float *ss = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
+                                        ((static_cast<size_t>(M) * D * 2 + 255) & ~static_cast<size_t>(255)));
+  return cuda_status(launch_out_proj(tmA, tmB, Y, ss, gain, x, h_out, M, D, K, eps, err_dev, as_stream(stream)));
+}
+
 size_t olmo3_attn_decode_workspace_size(int B, int H, int G, int d, int max_kv_len, int layer_type, int window,
                                         int num_splits) {
   if (B < 0 || H < 1 || G < 1 || !valid_d(d) || H % G != 0 || max_kv_len < 1 || !valid_type(layer_type) ||

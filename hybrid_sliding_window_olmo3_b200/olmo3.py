@@ -353,3 +353,37 @@ def qknorm_rope_yarn(q: torch.Tensor, k: torch.Tensor, gain_q: torch.Tensor, gai
                                         _p(v_out), _p(pos_offset), B, T, H, G, d, eps, theta, factor,
                                         original_context, beta_fast, beta_slow, _stream(stream)))
     return q_out, k_out, v_out
+
+
+def out_proj_workspace_size(M: int, D: int) -> int:
+    fn = lib().olmo3_out_proj_workspace_size
+    fn.argtypes = [_i, _i]
+    fn.restype = ctypes.c_size_t
+    return int(fn(M, D))
+
+
+def out_proj_postnorm_residual(attn: torch.Tensor, w_o: torch.Tensor, gain: torch.Tensor, x: torch.Tensor,
+                               h_out: Optional[torch.Tensor] = None, eps: float = 1e-6,
+                               workspace: Optional[torch.Tensor] = None, err: Optional[torch.Tensor] = None,
+                               stream=None):
+    """h = x + RMSNorm(attn W_o^T) * gain (output projection + reordered post-norm + residual)."""
+    fn = lib().olmo3_out_proj_postnorm_residual
+    fn.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, ctypes.c_float, _vp, ctypes.c_size_t, _vp, _vp]
+    fn.restype = _i
+    M, K = attn.shape
+    D = w_o.shape[0]
+    _dev(attn, "attn", torch.bfloat16)
+    _dev(w_o, "w_o", torch.bfloat16, (D, K))
+    _dev(gain, "gain", torch.float32, (D,))
+    _dev(x, "x", torch.bfloat16, (M, D))
+    if h_out is None:
+        h_out = torch.empty_like(x)
+    _dev(h_out, "h_out", torch.bfloat16, (M, D))
+    if err is not None:
+        _dev(err, "err", torch.int32)
+    if workspace is None:
+        workspace = torch.empty(max(out_proj_workspace_size(M, D), 16), dtype=torch.uint8, device=x.device)
+    _check("olmo3_out_proj_postnorm_residual",
+           fn(_p(attn), _p(w_o), _p(gain), _p(x), _p(h_out), M, D, K, eps, _p(workspace),
+              workspace.numel() * workspace.element_size(), _p(err), _stream(stream)))
+    return h_out

@@ -279,6 +279,25 @@ int olmo3_attn_decode_noalloc(const void *q, int H, const olmo3_kv_cache *c,
                               float *lse_out, float scale, int num_splits, int *err_dev,
                               void *stream);
 
+/*
+ * olmo3_out_proj_postnorm_residual - the attention block's output side: the
+ * bias-free output projection, then the reordered norm and the residual add
+ * ([CASE] ingredients 1 and 6, "Reordered norm": h = x + RMSNorm(Attention(x)),
+ * the norm acting on the projected attention output before the addition):
+ *     Y = attn W_o^T,   h = x + Y / sqrt(mean_j(Y_j^2) + eps) * gain.
+ *   attn    bf16 [M, K]: the attention output, heads side by side (K = H*d).
+ *   w_o     bf16 [D, K]: row j maps the attention features to model feature j.
+ *   gain    f32 [D];  x  bf16 [M, D] residual stream;  h_out bf16 [M, D] (may alias x).
+ *   workspace  olmo3_out_proj_workspace_size(M, D) bytes: Y in bf16, then the
+ *              per-row sums of squares (taken from the f32 products).
+ *   Requires K % 64 == 0 and D % 8 == 0.  The product runs on tcgen05 tensor cores
+ *   (128 x 256 tiles, f32 accumulation in tensor memory).
+ */
+size_t olmo3_out_proj_workspace_size(int M, int D);
+int olmo3_out_proj_postnorm_residual(const void *attn, const void *w_o, const float *gain,
+                                     const void *x, void *h_out, int M, int D, int K, float eps,
+                                     void *workspace, size_t ws_bytes, int *err_dev, void *stream);
+
 /* olmo3_status_string - a static English description of a status code. */
 const char *olmo3_status_string(int status);
 

@@ -165,6 +165,24 @@ def test_prefill_chunk_workspace_and_validation(lib):
     assert f(FAKE, FAKE, FAKE, ctypes.byref(c), FAKE, 0, 4, FAKE, 0.1, NULL, NULL, 0, NULL, NULL) == L.OK
 
 
+def test_out_proj_validation(lib):
+    assert L.out_proj_workspace_size(8192, 4096) == 8192 * 4096 * 2 + 8192 * 4
+    f = lib.olmo3_out_proj_postnorm_residual
+    f.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 3 + [ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t,
+                                                              ctypes.c_void_p, ctypes.c_void_p]
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, 16, 256, 128, 1e-6, FAKE, 1 << 20, NULL, NULL]
+    a = list(args); a[7] = 100                   # K not a multiple of 64
+    assert f(*a) == L.ERR_UNSUPPORTED
+    a = list(args); a[6] = 250                   # D not a multiple of 8
+    assert f(*a) == L.ERR_UNSUPPORTED
+    a = list(args); a[10] = 16                   # workspace too small
+    assert f(*a) == L.ERR_WORKSPACE
+    a = list(args); a[0] = NULL
+    assert f(*a) == L.ERR_INVALID_ARG
+    a = list(args); a[5] = 0                     # nothing to do
+    assert f(*a) == L.OK
+
+
 def test_mask_and_layer_types_reject_bad_arguments(lib):
     assert lib.olmo3_layer_types(-1, None) == L.ERR_INVALID_ARG
     assert lib.olmo3_layer_types(3, None) == L.ERR_INVALID_ARG

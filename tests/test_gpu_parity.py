@@ -444,6 +444,47 @@ def test_chunked_prefill_equals_one_shot(typ):
 
 
 # ---------------------------------------------------------------------------
+# Output side: projection + reordered post-norm + residual (tcgen05 GEMM)
+# ---------------------------------------------------------------------------
+def close_h(got, ref, n_ref, what=""):
+    """h = x + n is bf16 (one rounding of |h|) built from a bf16-rounded product (relative 2^-9 of |n|)."""
+    err = np.abs(got - ref)
+    bound = 2.0 ** -8 * (np.abs(ref) + np.abs(n_ref)) + 1e-3
+    assert (err <= bound).all(), f"{what}: {(err > bound).sum()} elements beyond the bound, worst {err.max():.3e}"
+
+
+@pytest.mark.parametrize("M,D,K", [(1, 256, 64), (100, 512, 128), (300, 4096, 4096), (130, 264, 192),
+                                   (257, 5120, 5120)])
+def test_out_proj_postnorm_residual_parity(M, D, K):
+    rng = np.random.default_rng(600 + M + D)
+    attn = bf16(rng.standard_normal((M, K)))
+    w = bf16(rng.standard_normal((D, K)) / np.sqrt(K))
+    x = bf16(rng.standard_normal((M, D)))
+    g = torch.from_numpy(rng.uniform(0.5, 1.5, D).astype(np.float32)).cuda()
+    err = new_err()
+    h = L.out_proj_postnorm_residual(attn, w, g, x, err=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    ref = O.out_proj_postnorm_residual(f64(x), f64(attn), f64(w), f64(g))
+    close_h(f64(h), ref, ref - f64(x), "out_proj")
+
+
+def test_out_proj_in_place_and_7b_sampled_rows():
+    rng = np.random.default_rng(9)
+    M, D, K = 8192, 4096, 4096
+    attn = WL.randn_bf16((M, K), 31, "cuda")
+    w = (WL.randn_bf16((D, K), 32, "cuda").float() / 64.0).to(torch.bfloat16)
+    x = WL.randn_bf16((M, D), 33, "cuda")
+    x0 = x.clone()
+    g = torch.rand(D, device="cuda") + 0.5
+    L.out_proj_postnorm_residual(attn, w, g, x, h_out=x)   # in place on the residual stream
+    torch.cuda.synchronize()
+    rows = sorted(set([0, 1, 127, 128, 4095, 8191] + rng.integers(0, M, 6).tolist()))
+    ref = O.out_proj_postnorm_residual(f64(x0[rows]), f64(attn[rows]), f64(w), f64(g))
+    close_h(f64(x[rows]), ref, ref - f64(x0[rows]), "out_proj 7B rows")
+
+
+# ---------------------------------------------------------------------------
 # The toy configuration end to end: 6 layers, prefill 16 tokens, 8 decode steps
 # ---------------------------------------------------------------------------
 def test_toy_pipeline_full_parity():
