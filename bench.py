@@ -610,6 +610,19 @@ def make_workload(name, dev, stream, batch=0, shared=False, chunk=0):
 
 
 # --------------------------------------------------------------------------
+def reduce_over_ranks(dist, dev, ms, work, ms_e2e, work_e2e):
+    """Replicas only: the step time is the slowest rank's, the work is the sum of
+    all ranks' (value = total work / max time).  Returns (ms_max, work_sum,
+    ms_e2e_max, work_e2e_sum); without a process group the rank's own figures."""
+    if dist is None:
+        return ms, work, ms_e2e, work_e2e
+    t = torch.tensor([ms, work, ms_e2e, work_e2e], dtype=torch.float64, device=dev)
+    tmax, tsum = t.clone(), t.clone()
+    dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
+    dist.all_reduce(tsum, op=dist.ReduceOp.SUM)
+    return tmax[0].item(), tsum[1].item(), tmax[2].item(), tsum[3].item()
+
+
 def run_ours(args):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -663,16 +676,8 @@ def run_ours(args):
         ms_e = f0.elapsed_time(f1)
         e2e = (work_e, ms_e)
 
-    t = torch.tensor([ms, work, e2e[1] if e2e else 0.0, e2e[0] if e2e else 0.0], dtype=torch.float64,
-                     device=dev)
-    if dist is not None:
-        tmax = t.clone()
-        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
-        tsum = t.clone()
-        dist.all_reduce(tsum, op=dist.ReduceOp.SUM)
-        ms_max, work_tot, ms_e_max, work_e_tot = tmax[0].item(), tsum[1].item(), tmax[2].item(), tsum[3].item()
-    else:
-        ms_max, work_tot, ms_e_max, work_e_tot = ms, work, t[2].item(), t[3].item()
+    ms_max, work_tot, ms_e_max, work_e_tot = reduce_over_ranks(
+        dist, dev, ms, work, e2e[1] if e2e else 0.0, e2e[0] if e2e else 0.0)
 
     if rank == 0:
         scale = 1.0  # TFLOP per ms*1e-3 -> TFLOP/s ; GB per s -> GB/s
