@@ -50,6 +50,7 @@ __all__ = [
     "rope", "qk_norm_rope", "attend", "prefill_attention", "KVCache",
     "append_slots", "decode_attention", "full_recompute_last_row", "chunk_attention",
     "yarn_inv_freq", "yarn_mscale", "rope_with", "qk_norm_rope_with", "out_proj_postnorm_residual",
+    "qkv_projection",
     "kv_bytes_per_token", "kv_cache_bytes",
 ]
 
@@ -258,6 +259,25 @@ def prefill_attention(q, k, v, layer_type: str, window: int,
         rows = np.arange(T)
     rows = np.asarray(rows)
     return attend(q[:, rows], pos[:, rows], k, pos, v, layer_type, window, scale)
+
+
+def qkv_projection(x, w_qkv, gain_q, gain_k, positions, H: int, G: int, d: int,
+                   eps: float = 1e-6, theta: float = 500000.0):
+    """[CASE] ingredient 1 (bias-free Q, K and V projections; the block's input x
+    is not normed first, ingredient 6) followed by ingredients 2 and 3.
+
+    x: [B, T, D]; w_qkv: [(H + 2G) d, D], rows of W_q, then W_k, then W_v;
+    positions [B, T].  Returns (q_hat [B, T, H, d], k_hat [B, T, G, d],
+    v [B, T, G, d]) in float64.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    B, T, _ = x.shape
+    y = np.einsum("btD,nD->btn", x, np.asarray(w_qkv, dtype=np.float64))
+    q = y[..., :H * d].reshape(B, T, H, d)
+    k = y[..., H * d:(H + G) * d].reshape(B, T, G, d)
+    v = y[..., (H + G) * d:].reshape(B, T, G, d)
+    qh, kh = qk_norm_rope(q, k, gain_q, gain_k, positions, eps, theta)
+    return qh, kh, v
 
 
 def out_proj_postnorm_residual(x, attn, w_o, gain, eps: float = 1e-6):

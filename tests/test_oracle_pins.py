@@ -403,6 +403,21 @@ def test_out_projection_is_a_plain_matmul():
     np.testing.assert_allclose(O.out_proj_postnorm_residual(x, a, w, np.ones(6)), ref, atol=1e-12)
 
 
+def test_qkv_projection_with_identity_weights_is_qknorm_rope_of_the_input():
+    rng = np.random.default_rng(15)
+    B, T, H, G, d = 2, 3, 4, 2, 8
+    D = (H + 2 * G) * d
+    x = rng.standard_normal((B, T, D))
+    gq, gk = rng.uniform(0.5, 1.5, H * d), rng.uniform(0.5, 1.5, G * d)
+    pos = np.array([[0, 1, 2], [40, 41, 42]])
+    qh, kh, v = O.qkv_projection(x, np.eye(D), gq, gk, pos, H, G, d)
+    rq, rk = O.qk_norm_rope(x[..., :H * d].reshape(B, T, H, d), x[..., H * d:(H + G) * d].reshape(B, T, G, d),
+                            gq, gk, pos)
+    np.testing.assert_allclose(qh, rq, atol=1e-12)
+    np.testing.assert_allclose(kh, rk, atol=1e-12)
+    np.testing.assert_allclose(v, x[..., (H + G) * d:].reshape(B, T, G, d), atol=0)
+
+
 def test_kv_sizing_matches_the_pages():
     g = {r[0]: float(r[1]) for r in read_golden("kv_sizing.txt")}
     t32 = O.layer_types(32)
