@@ -49,7 +49,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="7b-prefill",
                     choices=["7b-prefill", "32b-prefill", "7b-decode", "32b-decode", "ragged-7b-decode",
-                             "7b-prefill-chunked", "32b-prefill-chunked", "7b-out-proj", "32b-out-proj"])
+                             "7b-prefill-chunked", "32b-prefill-chunked", "7b-out-proj", "32b-out-proj",
+                             "7b-qkv-proj", "32b-qkv-proj"])
     ap.add_argument("--chunk", type=int, default=2048, help="prompt chunk of the *-prefill-chunked workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -518,7 +519,7 @@ class DecodeStep:
 
 class OutProjStep:
     """The attention block's output side for a whole prompt: h = x + RMSNorm(attn W_o^T) * gain
-    (tcgen05 GEMM with row sums of squares, then the norm + residual finisher)."""
+    (one persistent tcgen05 GEMM whose epilogue applies the row norm and the residual)."""
 
     def __init__(self, name, dev, stream):
         from hybrid_sliding_window_olmo3_b200 import olmo3 as L
@@ -541,11 +542,11 @@ class OutProjStep:
         self.ws = torch.empty(L.out_proj_workspace_size(M, D), dtype=torch.uint8, device=dev)
         self.flops = 2 * M * D * K
         self.unit = "TFLOP/s"
-        self.launches_per_step = 2  # GEMM + finisher (plus a memset of the row sums)
+        self.launches_per_step = 1  # the GEMM (plus a memset of the row sums and counters)
         self.h2d = sum(t.numel() * t.element_size() for t in self.host.values())
         self.d2h = M * D * 2
         self.ev = []
-        self.kernel_file, self.kernel_name = "out_proj.cu", "gemm_rowss_kernel + postnorm_residual_kernel"
+        self.kernel_file, self.kernel_name = "proj_gemm.cu", "proj_gemm_kernel<PostNormEpilogue>"
         self.config = {"workload": f"OLMo 3 {sh.name[6:]} attention output side: h = x + RMSNorm(attn W_o^T), "
                                    f"M={M} tokens, K={K}, D={D}, bf16",
                        "global_batch": wl.B, "seq_len": wl.T, "l2": "inputs larger than L2", "parallelism": "replicas"}
@@ -599,7 +600,90 @@ class OutProjStep:
                 "sample": f"{rows} rows (fp64 matmul with W_o, norm, residual), {el:.1f} s; numpy (BLAS threads)"}
 
 
+class QkvProjStep(OutProjStep):
+    """The attention block's input side for a whole prompt: [q|k|v] = x W_qkv^T, then QK-norm
+    + RoPE on q and k (one persistent tcgen05 GEMM with the norm and rotation in its epilogue)."""
+
+    def __init__(self, name, dev, stream):
+        from hybrid_sliding_window_olmo3_b200 import olmo3 as L
+        from hybrid_sliding_window_olmo3_b200 import workloads as WL
+        self.L = L
+        wl = WL.WORKLOADS[name.replace("qkv-proj", "prefill")]
+        sh = wl.shape
+        self.sh, self.dev, self.stream, self.wl = sh, dev, stream, wl
+        D = {"olmo3-7b": 4096, "olmo3-32b": 5120}[sh.name]
+        M, N = wl.B * wl.T, (sh.H + 2 * sh.G) * sh.d
+        self.M, self.D, self.K, self.N = M, N, D, N
+        host = dict(x=WL.randn_bf16((wl.B, wl.T, D), wl.seed + 21),
+                    w=(WL.randn_bf16((N, D), wl.seed + 22).float() / D ** 0.5).to(torch.bfloat16),
+                    gq=torch.rand(sh.H * sh.d, generator=torch.Generator().manual_seed(wl.seed + 23)) + 0.5,
+                    gk=torch.rand(sh.G * sh.d, generator=torch.Generator().manual_seed(wl.seed + 24)) + 0.5,
+                    pos=torch.zeros(wl.B, dtype=torch.int32))
+        self.host = {n: t.pin_memory() for n, t in host.items()}
+        for n, t in host.items():
+            setattr(self, n, t.to(dev))
+        B, T = wl.B, wl.T
+        self.outs = (torch.empty(B, T, sh.H, sh.d, dtype=torch.bfloat16, device=dev),
+                     torch.empty(B, T, sh.G, sh.d, dtype=torch.bfloat16, device=dev),
+                     torch.empty(B, T, sh.G, sh.d, dtype=torch.bfloat16, device=dev))
+        self.outs_host = tuple(torch.empty(o.shape, dtype=torch.bfloat16).pin_memory() for o in self.outs)
+        self.ws = torch.empty(L.qkv_proj_workspace_size(M), dtype=torch.uint8, device=dev)
+        self.flops = 2 * M * N * D
+        self.unit = "TFLOP/s"
+        self.launches_per_step = 1  # the GEMM (plus a memset of the row sums and counters)
+        self.h2d = sum(t.numel() * t.element_size() for t in self.host.values())
+        self.d2h = M * N * 2
+        self.ev = []
+        self.kernel_file, self.kernel_name = "proj_gemm.cu", "proj_gemm_kernel<QkvEpilogue<128>>"
+        self.config = {"workload": f"OLMo 3 {sh.name[6:]} attention input side: [q|k|v] = x W_qkv^T + QK-norm + "
+                                   f"RoPE, M={M} tokens, D={D}, N={N} (H={sh.H}, G={sh.G}, d={sh.d}), bf16",
+                       "global_batch": wl.B, "seq_len": wl.T, "l2": "inputs larger than L2", "parallelism": "replicas"}
+
+    def step(self, timed_kernel=False, host_io=False):
+        s, sh = self.stream, self.sh
+        if host_io:
+            for n in ("x", "w", "gq", "gk", "pos"):
+                getattr(self, n).copy_(self.host[n], non_blocking=True)
+        if timed_kernel:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+        q, k, v = self.outs
+        self.L.qkv_proj_qknorm_rope(self.x, self.w, self.gq, self.gk, self.pos, sh.H, sh.G, sh.d, theta=sh.theta,
+                                    q_out=q, k_out=k, v_out=v, workspace=self.ws, stream=s)
+        if timed_kernel:
+            e1.record(s)
+            self.ev.append((e0, e1, self.flops))
+        if host_io:
+            for o, h in zip(self.outs, self.outs_host):
+                h.copy_(o, non_blocking=True)
+
+    def cpu_baseline(self, seconds):
+        import oracle.olmo3_oracle as O
+        sh = self.sh
+        x, w, gq, gk = (self.host[n].float().numpy() for n in ("x", "w", "gq", "gk"))
+        x = x.reshape(self.M, self.K)
+        done, el, rows = 0, 0.0, 0
+        rng = np.random.default_rng(0)
+        while el < seconds:
+            r = rng.integers(0, self.M, 8)
+            pos = (r % self.wl.T)[None]
+            t0 = time.perf_counter()
+            O.qkv_projection(x[r][None], w, gq, gk, pos, sh.H, sh.G, sh.d, theta=sh.theta)
+            el += time.perf_counter() - t0
+            done += 2 * 8 * self.N * self.K
+            rows += 8
+        try:
+            from threadpoolctl import threadpool_info
+            cores = max([i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"] or [1])
+        except Exception:  # noqa: BLE001 - reporting only
+            cores = len(os.sched_getaffinity(0))
+        return {"value": done / el / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                "sample": f"{rows} rows (fp64 matmul with W_qkv, QK-norm, RoPE), {el:.1f} s; numpy (BLAS threads)"}
+
+
 def make_workload(name, dev, stream, batch=0, shared=False, chunk=0):
+    if name.endswith("qkv-proj"):
+        return QkvProjStep(name, dev, stream)
     if name.endswith("out-proj"):
         return OutProjStep(name, dev, stream)
     if name.endswith("prefill"):

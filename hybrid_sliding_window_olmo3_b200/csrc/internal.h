@@ -64,9 +64,26 @@ cudaError_t launch_gather_window(const olmo3_kv_cache &c, const void *k_new, con
                                  const int32_t *pos_offset, int T, int Tk, void *k_out, void *v_out,
                                  cudaStream_t stream);
 
-// Y = A B^T (tcgen05) with per-row sums of squares, then h = x + Y rsqrt(ss/N + eps) gain.
-// tmA: 2-d map over A [M, K] with 64 x 128 boxes; tmB: over B [N, K] with 64 x 256 boxes.
-cudaError_t launch_out_proj(const CUtensorMap &tmA, const CUtensorMap &tmB, void *Y, float *ss, const float *gain,
-                            const void *x, void *h, int M, int N, int K, float eps, int *err, cudaStream_t stream);
+// Persistent tcgen05 GEMMs with the row norm fused into the epilogue (proj_gemm.cu).
+// A norm group (the q or the k columns of a row, or a whole Wo row) may span at
+// most proj_gemm_max_tiles_per_row() 256-column tiles.  The workspace starts with proj_gemm_flags_bytes(M, groups) bytes that the
+// launcher zeroes (per-row sums of squares and per-row-block counters; groups = 2
+// for q and k, 1 for Wo).
+int proj_gemm_max_tiles_per_row();
+size_t proj_gemm_flags_bytes(int M, int groups);
+constexpr int kProjTileN = 256;
+
+// q, k, v = split(X W^T); q, k <- RoPE(RMSNorm(.)) as in launch_qknorm_rope.
+// tmX: 2-d map over X [B*T, Dm] with 64 x 128 boxes; tmW over W [(H+2G) d, Dm] with
+// 64 x 256 boxes (both 128-byte swizzle).  Requires H*d and G*d multiples of 256.
+cudaError_t launch_qkv_proj(const CUtensorMap &tmX, const CUtensorMap &tmW, void *q, void *k, void *v,
+                            const float *gain_q, const float *gain_k, const int32_t *pos_offset, int B, int T, int H,
+                            int G, int d, int Dm, float eps, const RopeTable &tab, void *ws, int *err,
+                            cudaStream_t stream);
+
+// h = x + (A B^T) rsqrt(rowmean((A B^T)^2) + eps) gain.  tmA: 2-d map over A [M, K]
+// with 64 x 128 boxes; tmB: over B [N, K] with 64 x 256 boxes.
+cudaError_t launch_out_proj(const CUtensorMap &tmA, const CUtensorMap &tmB, const float *gain, const void *x, void *h,
+                            int M, int N, int K, float eps, void *ws, int *err, cudaStream_t stream);
 
 }  // namespace olmo3

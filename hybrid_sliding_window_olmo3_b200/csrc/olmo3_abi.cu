@@ -103,6 +103,40 @@ int olmo3_attn_mask(int T, int window, int layer_type, uint8_t *out_dev, void *s
 }
 
 namespace {
+// NTK-by-parts: pair i turns r = original_context * f_i / (2 pi) times over the
+// original context; it keeps f_i when r >= beta_fast, becomes f_i / factor when
+// r <= beta_slow, and blends linearly in between.  factor 1 is plain RoPE.
+bool yarn_table(int d, double theta, double factor, int original_context, double beta_fast, double beta_slow,
+                RopeTable *tab) {
+  if (!(theta > 0.0) || !(factor >= 1.0) || original_context < 1 || !(beta_fast > beta_slow)) return false;
+  const double two_pi = 6.283185307179586476925286766559;
+  for (int i = 0; i < 64; ++i) {
+    if (i >= d / 2) {
+      tab->inv_freq[i] = 0.0;
+      continue;
+    }
+    const double f = pow(theta, -2.0 * i / d);
+    if (factor == 1.0) {
+      tab->inv_freq[i] = f;
+      continue;
+    }
+    const double r = original_context * f / two_pi;
+    double keep = (r - beta_slow) / (beta_fast - beta_slow);
+    keep = keep < 0.0 ? 0.0 : (keep > 1.0 ? 1.0 : keep);
+    tab->inv_freq[i] = f * keep + (f / factor) * (1.0 - keep);
+  }
+  tab->out_scale = factor > 1.0 ? static_cast<float>(0.1 * log(factor) + 1.0) : 1.0f;
+  return true;
+}
+
+// The persistent projection GEMMs need every tile of a 128-row block resident at
+// once: at most one SM's worth of tiles per row.
+int tiles_per_row_status(int tiles) {
+  const int max_tiles = proj_gemm_max_tiles_per_row();
+  if (max_tiles <= 0) return OLMO3_ERR_CUDA;
+  return tiles > max_tiles ? OLMO3_ERR_UNSUPPORTED : OLMO3_OK;
+}
+
 int qknorm_rope_common(const void *q, const void *k, const void *v, int in_dtype, const float *gain_q,
                        const float *gain_k, void *q_out, void *k_out, void *v_out, const int32_t *pos_offset, int B,
                        int T, int H, int G, int d, float eps, const RopeTable &tab, void *stream) {
@@ -138,29 +172,8 @@ int olmo3_qknorm_rope_yarn(const void *q, const void *k, const void *v, int in_d
                            const float *gain_k, void *q_out, void *k_out, void *v_out, const int32_t *pos_offset,
                            int B, int T, int H, int G, int d, float eps, double theta, double factor,
                            int original_context, double beta_fast, double beta_slow, void *stream) {
-  if (!(theta > 0.0) || !(factor >= 1.0) || original_context < 1 || !(beta_fast > beta_slow))
-    return OLMO3_ERR_INVALID_ARG;
-  // NTK-by-parts: pair i turns r = original_context * f_i / (2 pi) times over the
-  // original context; it keeps f_i when r >= beta_fast, becomes f_i / factor when
-  // r <= beta_slow, and blends linearly in between.
   RopeTable tab;
-  const double two_pi = 6.283185307179586476925286766559;
-  for (int i = 0; i < 64; ++i) {
-    if (i >= d / 2) {
-      tab.inv_freq[i] = 0.0;
-      continue;
-    }
-    const double f = pow(theta, -2.0 * i / d);
-    if (factor == 1.0) {
-      tab.inv_freq[i] = f;
-      continue;
-    }
-    const double r = original_context * f / two_pi;
-    double keep = (r - beta_slow) / (beta_fast - beta_slow);
-    keep = keep < 0.0 ? 0.0 : (keep > 1.0 ? 1.0 : keep);
-    tab.inv_freq[i] = f * keep + (f / factor) * (1.0 - keep);
-  }
-  tab.out_scale = factor > 1.0 ? static_cast<float>(0.1 * log(factor) + 1.0) : 1.0f;
+  if (!yarn_table(d, theta, factor, original_context, beta_fast, beta_slow, &tab)) return OLMO3_ERR_INVALID_ARG;
   return qknorm_rope_common(q, k, v, in_dtype, gain_q, gain_k, q_out, k_out, v_out, pos_offset, B, T, H, G, d, eps,
                             tab, stream);
 }
@@ -245,16 +258,15 @@ int olmo3_attn_prefill_chunk(const void *q, const void *k_new, const void *v_new
 
 size_t olmo3_out_proj_workspace_size(int M, int D) {
   if (M < 0 || D < 1) return 0;
-  const size_t y = (static_cast<size_t>(M) * D * 2 + 255) & ~static_cast<size_t>(255);
-  return y + static_cast<size_t>(M) * 4;
+  return (proj_gemm_flags_bytes(M, 1) + 255) & ~static_cast<size_t>(255);
 }
 
 int olmo3_out_proj_postnorm_residual(const void *attn, const void *w_o, const float *gain, const void *x, void *h_out,
                                      int M, int D, int K, float eps, void *workspace, size_t ws_bytes, int *err_dev,
                                      void *stream) {
+  int st = OLMO3_OK;
   if (M < 0 || D < 1 || K < 1 || !(eps >= 0.f)) return OLMO3_ERR_INVALID_ARG;
-  if (K % 64 != 0 || D % 8 != 0 || M > 65535 * 128 || static_cast<int64_t>(M) * D >= (int64_t(1) << 31))
-    return OLMO3_ERR_UNSUPPORTED;
+  if (K % 64 != 0 || D % 8 != 0 || static_cast<int64_t>(M) * D >= (int64_t(1) << 31)) return OLMO3_ERR_UNSUPPORTED;
   if (M == 0) return OLMO3_OK;
   if (!attn || !w_o || !gain || !x || !h_out) return OLMO3_ERR_INVALID_ARG;
   const void *ptrs[] = {attn, w_o, gain, x, h_out};
@@ -262,6 +274,8 @@ int olmo3_out_proj_postnorm_residual(const void *attn, const void *w_o, const fl
     if (!aligned16(p)) return OLMO3_ERR_INVALID_ARG;
   const size_t need = olmo3_out_proj_workspace_size(M, D);
   if (workspace == nullptr || ws_bytes < need || !aligned16(workspace)) return OLMO3_ERR_WORKSPACE;
+  st = tiles_per_row_status((D + kProjTileN - 1) / kProjTileN);
+  if (st != OLMO3_OK) return st;
   CUtensorMap tmA, tmB;
   const cuuint32_t box_a[2] = {64, 128}, box_b[2] = {64, 256};
   const cuuint64_t dims_a[2] = {(cuuint64_t)K, (cuuint64_t)M}, dims_b[2] = {(cuuint64_t)K, (cuuint64_t)D};
@@ -269,10 +283,45 @@ int olmo3_out_proj_postnorm_residual(const void *attn, const void *w_o, const fl
   if (!encode_bf16(&tmA, attn, 2, dims_a, stride, box_a, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_bf16(&tmB, w_o, 2, dims_b, stride, box_b, CU_TENSOR_MAP_SWIZZLE_128B))
     return OLMO3_ERR_CUDA;
-  void *Y = workspace;
-  float *ss = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
-                                        ((static_cast<size_t>(M) * D * 2 + 255) & ~static_cast<size_t>(255)));
-  return cuda_status(launch_out_proj(tmA, tmB, Y, ss, gain, x, h_out, M, D, K, eps, err_dev, as_stream(stream)));
+  return cuda_status(launch_out_proj(tmA, tmB, gain, x, h_out, M, D, K, eps, workspace, err_dev, as_stream(stream)));
+}
+
+size_t olmo3_qkv_proj_workspace_size(int M) {
+  if (M < 0) return 0;
+  return (proj_gemm_flags_bytes(M, 2) + 255) & ~static_cast<size_t>(255);
+}
+
+int olmo3_qkv_proj_qknorm_rope(const void *x, const void *w_qkv, const float *gain_q, const float *gain_k,
+                               void *q_out, void *k_out, void *v_out, const int32_t *pos_offset, int B, int T, int H,
+                               int G, int d, int D, float eps, double theta, double rope_factor, int original_context,
+                               double beta_fast, double beta_slow, void *workspace, size_t ws_bytes, int *err_dev,
+                               void *stream) {
+  if (B < 0 || T < 0 || H < 1 || G < 1 || D < 1 || !(eps >= 0.f)) return OLMO3_ERR_INVALID_ARG;
+  RopeTable tab;
+  if (!yarn_table(d, theta, rope_factor, original_context, beta_fast, beta_slow, &tab)) return OLMO3_ERR_INVALID_ARG;
+  if (!valid_d(d) || D % 64 != 0 || (H * d) % kProjTileN != 0 || (G * d) % kProjTileN != 0)
+    return OLMO3_ERR_UNSUPPORTED;
+  const int64_t M = static_cast<int64_t>(B) * T;
+  const int64_t N = static_cast<int64_t>(H + 2 * G) * d;
+  if (M * (D > N ? D : N) >= (int64_t(1) << 31)) return OLMO3_ERR_UNSUPPORTED;
+  if (M == 0) return OLMO3_OK;
+  if (!x || !w_qkv || !gain_q || !gain_k || !q_out || !k_out || !v_out || !pos_offset) return OLMO3_ERR_INVALID_ARG;
+  const void *ptrs[] = {x, w_qkv, gain_q, gain_k, q_out, k_out, v_out};
+  for (const void *p : ptrs)
+    if (!aligned16(p)) return OLMO3_ERR_INVALID_ARG;
+  const size_t need = olmo3_qkv_proj_workspace_size(static_cast<int>(M));
+  if (workspace == nullptr || ws_bytes < need || !aligned16(workspace)) return OLMO3_ERR_WORKSPACE;
+  const int st = tiles_per_row_status((H > G ? H : G) * d / kProjTileN);
+  if (st != OLMO3_OK) return st;
+  CUtensorMap tmX, tmW;
+  const cuuint32_t box_x[2] = {64, 128}, box_w[2] = {64, 256};
+  const cuuint64_t dims_x[2] = {(cuuint64_t)D, (cuuint64_t)M}, dims_w[2] = {(cuuint64_t)D, (cuuint64_t)N};
+  const cuuint64_t stride[1] = {(cuuint64_t)D * 2};
+  if (!encode_bf16(&tmX, x, 2, dims_x, stride, box_x, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_bf16(&tmW, w_qkv, 2, dims_w, stride, box_w, CU_TENSOR_MAP_SWIZZLE_128B))
+    return OLMO3_ERR_CUDA;
+  return cuda_status(launch_qkv_proj(tmX, tmW, q_out, k_out, v_out, gain_q, gain_k, pos_offset, B, T, H, G, d, D, eps,
+                                     tab, workspace, err_dev, as_stream(stream)));
 }
 
 size_t olmo3_attn_decode_workspace_size(int B, int H, int G, int d, int max_kv_len, int layer_type, int window,

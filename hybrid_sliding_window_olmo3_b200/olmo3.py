@@ -387,3 +387,44 @@ def out_proj_postnorm_residual(attn: torch.Tensor, w_o: torch.Tensor, gain: torc
            fn(_p(attn), _p(w_o), _p(gain), _p(x), _p(h_out), M, D, K, eps, _p(workspace),
               workspace.numel() * workspace.element_size(), _p(err), _stream(stream)))
     return h_out
+
+
+def qkv_proj_workspace_size(M: int) -> int:
+    fn = lib().olmo3_qkv_proj_workspace_size
+    fn.argtypes = [_i]
+    fn.restype = ctypes.c_size_t
+    return int(fn(M))
+
+
+def qkv_proj_qknorm_rope(x: torch.Tensor, w_qkv: torch.Tensor, gain_q: torch.Tensor, gain_k: torch.Tensor,
+                         pos_offset: torch.Tensor, H: int, G: int, d: int, eps: float = 1e-6,
+                         theta: float = 500000.0, factor: float = 1.0, original_context: int = 8192,
+                         beta_fast: float = 32.0, beta_slow: float = 1.0, q_out=None, k_out=None, v_out=None,
+                         workspace: Optional[torch.Tensor] = None, err: Optional[torch.Tensor] = None, stream=None):
+    """[q | k | v] = x W_qkv^T, then QK-norm + RoPE (YaRN when factor > 1) on q and k, in one kernel."""
+    fn = lib().olmo3_qkv_proj_qknorm_rope
+    fn.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, ctypes.c_float,
+                   ctypes.c_double, ctypes.c_double, _i, ctypes.c_double, ctypes.c_double, _vp, ctypes.c_size_t,
+                   _vp, _vp]
+    fn.restype = _i
+    B, T, D = x.shape
+    _dev(x, "x", torch.bfloat16)
+    _dev(w_qkv, "w_qkv", torch.bfloat16, ((H + 2 * G) * d, D))
+    _dev(gain_q, "gain_q", torch.float32, (H * d,))
+    _dev(gain_k, "gain_k", torch.float32, (G * d,))
+    _dev(pos_offset, "pos_offset", torch.int32, (B,))
+    q_out = torch.empty((B, T, H, d), dtype=torch.bfloat16, device=x.device) if q_out is None else q_out
+    k_out = torch.empty((B, T, G, d), dtype=torch.bfloat16, device=x.device) if k_out is None else k_out
+    v_out = torch.empty((B, T, G, d), dtype=torch.bfloat16, device=x.device) if v_out is None else v_out
+    _dev(q_out, "q_out", torch.bfloat16, (B, T, H, d))
+    _dev(k_out, "k_out", torch.bfloat16, (B, T, G, d))
+    _dev(v_out, "v_out", torch.bfloat16, (B, T, G, d))
+    if err is not None:
+        _dev(err, "err", torch.int32)
+    if workspace is None:
+        workspace = torch.empty(max(qkv_proj_workspace_size(B * T), 16), dtype=torch.uint8, device=x.device)
+    _check("olmo3_qkv_proj_qknorm_rope",
+           fn(_p(x), _p(w_qkv), _p(gain_q), _p(gain_k), _p(q_out), _p(k_out), _p(v_out), _p(pos_offset), B, T, H, G,
+              d, D, eps, theta, factor, original_context, beta_fast, beta_slow, _p(workspace),
+              workspace.numel() * workspace.element_size(), _p(err), _stream(stream)))
+    return q_out, k_out, v_out

@@ -288,15 +288,48 @@ int olmo3_attn_decode_noalloc(const void *q, int H, const olmo3_kv_cache *c,
  *   attn    bf16 [M, K]: the attention output, heads side by side (K = H*d).
  *   w_o     bf16 [D, K]: row j maps the attention features to model feature j.
  *   gain    f32 [D];  x  bf16 [M, D] residual stream;  h_out bf16 [M, D] (may alias x).
- *   workspace  olmo3_out_proj_workspace_size(M, D) bytes: Y in bf16, then the
- *              per-row sums of squares (taken from the f32 products).
- *   Requires K % 64 == 0 and D % 8 == 0.  The product runs on tcgen05 tensor cores
- *   (128 x 256 tiles, f32 accumulation in tensor memory).
+ *   workspace  olmo3_out_proj_workspace_size(M, D) bytes (per-row sums of squares and
+ *              per-row-block counters; zeroed by the call itself).
+ *   err_dev    optional device int; OLMO3_DEVERR_TIMEOUT is or-ed in when a wait gave up.
+ *   Requires K % 64 == 0, D % 8 == 0 and D <= 256 * (SM count).  One persistent
+ *   kernel on tcgen05 tensor cores (128 x 256 tiles, f32 accumulation in tensor
+ *   memory): the norm of a row needs all of its D features, which span several
+ *   tiles, so each tile publishes its share of the row sums, waits (bounded) for
+ *   the other tiles of its 128 rows, then writes h; Y never goes to HBM.
  */
 size_t olmo3_out_proj_workspace_size(int M, int D);
 int olmo3_out_proj_postnorm_residual(const void *attn, const void *w_o, const float *gain,
                                      const void *x, void *h_out, int M, int D, int K, float eps,
                                      void *workspace, size_t ws_bytes, int *err_dev, void *stream);
+
+/*
+ * olmo3_qkv_proj_qknorm_rope - the attention block's input side in one kernel:
+ * the bias-free Q, K and V projections of the block input ([CASE] ingredient 1;
+ * ingredient 6 leaves that input un-normed), then QK-norm and RoPE on q and k
+ * exactly as olmo3_qknorm_rope_yarn (plain RoPE when rope_factor == 1):
+ *     [q | k | v] = x W_qkv^T,  q <- RoPE(RMSNorm_{H*d}(q) gain_q),  k likewise over G*d.
+ *   x       bf16 [B, T, D] (D = model width; rows b*T + t).
+ *   w_qkv   bf16 [(H + 2G) d, D]: rows of W_q (H*d), then W_k (G*d), then W_v (G*d).
+ *   gain_q  f32 [H*d];  gain_k  f32 [G*d];  pos_offset int32 [B] as olmo3_qknorm_rope.
+ *   q_out   bf16 [B, T, H, d];  k_out, v_out  bf16 [B, T, G, d]; none may alias x.
+ *   theta, rope_factor, original_context, beta_fast, beta_slow: as olmo3_qknorm_rope_yarn.
+ *   workspace  olmo3_qkv_proj_workspace_size(B*T) bytes, 16-byte aligned (per-row
+ *              sums of squares of q and k, per-row-block counters; zeroed by the call).
+ *   err_dev    optional device int; OLMO3_DEVERR_TIMEOUT is or-ed in when a wait gave up.
+ *   Requires d in {64, 128}, D % 64 == 0, H*d and G*d multiples of 256, and
+ *   H*d, G*d <= 256 * (SM count); OLMO3_ERR_UNSUPPORTED otherwise.
+ *   One persistent tcgen05 kernel (128 x 256 tiles): the epilogue applies the gains
+ *   and the rotation to the f32 accumulator, and the per-row RMSNorm factor (which
+ *   needs the sums over all q or all k tiles of the row) once every tile of the
+ *   row's 128-row block has published its share.
+ */
+size_t olmo3_qkv_proj_workspace_size(int M);
+int olmo3_qkv_proj_qknorm_rope(const void *x, const void *w_qkv, const float *gain_q,
+                               const float *gain_k, void *q_out, void *k_out, void *v_out,
+                               const int32_t *pos_offset, int B, int T, int H, int G, int d,
+                               int D, float eps, double theta, double rope_factor,
+                               int original_context, double beta_fast, double beta_slow,
+                               void *workspace, size_t ws_bytes, int *err_dev, void *stream);
 
 /* olmo3_status_string - a static English description of a status code. */
 const char *olmo3_status_string(int status);

@@ -262,21 +262,25 @@ def prefill_attention(q, k, v, layer_type: str, window: int,
 
 
 def qkv_projection(x, w_qkv, gain_q, gain_k, positions, H: int, G: int, d: int,
-                   eps: float = 1e-6, theta: float = 500000.0):
+                   eps: float = 1e-6, theta: float = 500000.0, inv_freq=None, out_scale: float = 1.0):
     """[CASE] ingredient 1 (bias-free Q, K and V projections; the block's input x
     is not normed first, ingredient 6) followed by ingredients 2 and 3.
 
     x: [B, T, D]; w_qkv: [(H + 2G) d, D], rows of W_q, then W_k, then W_v;
-    positions [B, T].  Returns (q_hat [B, T, H, d], k_hat [B, T, G, d],
-    v [B, T, G, d]) in float64.
+    positions [B, T].  inv_freq / out_scale, when given, replace plain RoPE
+    (YaRN on full layers, see qk_norm_rope_with).  Returns (q_hat [B, T, H, d],
+    k_hat [B, T, G, d], v [B, T, G, d]) in float64.
     """
     x = np.asarray(x, dtype=np.float64)
     B, T, _ = x.shape
-    y = np.einsum("btD,nD->btn", x, np.asarray(w_qkv, dtype=np.float64))
+    y = x @ np.asarray(w_qkv, dtype=np.float64).T
     q = y[..., :H * d].reshape(B, T, H, d)
     k = y[..., H * d:(H + G) * d].reshape(B, T, G, d)
     v = y[..., (H + G) * d:].reshape(B, T, G, d)
-    qh, kh = qk_norm_rope(q, k, gain_q, gain_k, positions, eps, theta)
+    if inv_freq is None:
+        qh, kh = qk_norm_rope(q, k, gain_q, gain_k, positions, eps, theta)
+    else:
+        qh, kh = qk_norm_rope_with(q, k, gain_q, gain_k, positions, inv_freq, out_scale, eps)
     return qh, kh, v
 
 

@@ -166,7 +166,8 @@ def test_prefill_chunk_workspace_and_validation(lib):
 
 
 def test_out_proj_validation(lib):
-    assert L.out_proj_workspace_size(8192, 4096) == 8192 * 4096 * 2 + 8192 * 4
+    # per-row sums of squares, one counter per 128-row block and an abort flag, in 256-byte units
+    assert L.out_proj_workspace_size(8192, 4096) == (8192 * 4 + (64 + 1) * 4 + 255) // 256 * 256
     f = lib.olmo3_out_proj_postnorm_residual
     f.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 3 + [ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t,
                                                               ctypes.c_void_p, ctypes.c_void_p]
@@ -180,6 +181,38 @@ def test_out_proj_validation(lib):
     a = list(args); a[0] = NULL
     assert f(*a) == L.ERR_INVALID_ARG
     a = list(args); a[5] = 0                     # nothing to do
+    assert f(*a) == L.OK
+
+
+def test_qkv_proj_validation(lib):
+    # q and k sums of squares per row, two counters per 128-row block and an abort flag
+    assert L.qkv_proj_workspace_size(8192) == (8192 * 8 + (2 * 64 + 1) * 4 + 255) // 256 * 256
+    assert L.qkv_proj_workspace_size(0) == 256
+    f = lib.olmo3_qkv_proj_qknorm_rope
+    d_ = ctypes.c_double
+    f.argtypes = [ctypes.c_void_p] * 8 + [ctypes.c_int] * 6 + [ctypes.c_float, d_, d_, ctypes.c_int, d_, d_,
+                                                               ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+                                                               ctypes.c_void_p]
+    #       x     w     gq    gk    q     k     v     pos   B  T   H  G  d    D    eps   theta factor oc   bf  bs
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 50, 4, 2, 128, 256, 1e-6, 5e5, 1.0, 8192, 32., 1.,
+            FAKE, 1 << 20, NULL, NULL]
+    a = list(args); a[12] = 96                   # head dim
+    assert f(*a) == L.ERR_UNSUPPORTED
+    a = list(args); a[13] = 200                  # model width not a multiple of 64
+    assert f(*a) == L.ERR_UNSUPPORTED
+    a = list(args); a[10], a[11] = 3, 1          # H*d not a multiple of 256
+    assert f(*a) == L.ERR_UNSUPPORTED
+    a = list(args); a[11], a[10] = 1, 4          # G*d = 128
+    assert f(*a) == L.ERR_UNSUPPORTED
+    a = list(args); a[16] = 0.5                  # YaRN factor below 1
+    assert f(*a) == L.ERR_INVALID_ARG
+    a = list(args); a[15] = 0.0                  # theta
+    assert f(*a) == L.ERR_INVALID_ARG
+    a = list(args); a[21] = 64                   # workspace too small
+    assert f(*a) == L.ERR_WORKSPACE
+    a = list(args); a[7] = NULL                  # no positions
+    assert f(*a) == L.ERR_INVALID_ARG
+    a = list(args); a[9] = 0                     # nothing to do
     assert f(*a) == L.OK
 
 

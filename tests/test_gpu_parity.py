@@ -447,7 +447,9 @@ def test_chunked_prefill_equals_one_shot(typ):
 # Output side: projection + reordered post-norm + residual (tcgen05 GEMM)
 # ---------------------------------------------------------------------------
 def close_h(got, ref, n_ref, what=""):
-    """h = x + n is bf16 (one rounding of |h|) built from a bf16-rounded product (relative 2^-9 of |n|)."""
+    """h = x + n is rounded once to bf16 (2^-9 |h|); n comes from an f32 product and
+    an f32 norm.  The bar allows 2^-8 of |h| + |n| (twice the rounding, plus room
+    for the f32 accumulation over K) and 1e-3 absolute."""
     err = np.abs(got - ref)
     bound = 2.0 ** -8 * (np.abs(ref) + np.abs(n_ref)) + 1e-3
     assert (err <= bound).all(), f"{what}: {(err > bound).sum()} elements beyond the bound, worst {err.max():.3e}"
@@ -482,6 +484,107 @@ def test_out_proj_in_place_and_7b_sampled_rows():
     rows = sorted(set([0, 1, 127, 128, 4095, 8191] + rng.integers(0, M, 6).tolist()))
     ref = O.out_proj_postnorm_residual(f64(x0[rows]), f64(attn[rows]), f64(w), f64(g))
     close_h(f64(x[rows]), ref, ref - f64(x0[rows]), "out_proj 7B rows")
+
+
+# ---------------------------------------------------------------------------
+# Input side: fused QKV projection + QK-norm + RoPE (persistent tcgen05 GEMM)
+# ---------------------------------------------------------------------------
+def qkv_inputs(B, T, H, G, d, D, seed):
+    rng = np.random.default_rng(seed)
+    x = bf16(rng.standard_normal((B, T, D)))
+    w = bf16(rng.standard_normal(((H + 2 * G) * d, D)) / np.sqrt(D))
+    gq = torch.from_numpy(rng.uniform(0.5, 1.5, H * d).astype(np.float32)).cuda()
+    gk = torch.from_numpy(rng.uniform(0.5, 1.5, G * d).astype(np.float32)).cuda()
+    return x, w, gq, gk
+
+
+def check_qkv(got, x, w, gq, gk, offs, H, G, d, rows=None, yarn=None, what=""):
+    """q and k within bf16 rounding of the oracle (f32 accumulation adds far less);
+    v likewise (one rounding of an f32 sum)."""
+    B, T, D = x.shape
+    xs, qo, ko, vo = f64(x), f64(got[0]), f64(got[1]), f64(got[2])
+    pos = np.asarray(offs)[:, None] + np.arange(T)[None, :]
+    kw = {}
+    if yarn is not None:
+        kw = dict(inv_freq=O.yarn_inv_freq(d, 5e5, yarn, 8192), out_scale=O.yarn_mscale(yarn))
+    if rows is not None:  # sampled tokens (b, t)
+        bi, ti = np.array([r[0] for r in rows]), np.array([r[1] for r in rows])
+        xs, pos = xs[bi, ti][None], pos[bi, ti][None]
+        qo, ko, vo = qo[bi, ti][None], ko[bi, ti][None], vo[bi, ti][None]
+    rq, rk, rv = O.qkv_projection(xs, f64(w), f64(gq), f64(gk), pos, H, G, d, **kw)
+    close_qk(qo, rq, what + " q")
+    close_qk(ko, rk, what + " k")
+    close_qk(vo, rv, what + " v")
+
+
+@pytest.mark.parametrize("B,T,H,G,d,D,offs", [
+    (1, 1, 2, 2, 128, 64, [0]),              # one row, one K slice, one tile each of q, k, v
+    (2, 100, 4, 2, 128, 256, [0, 37]),       # ragged second row block, position offsets
+    (3, 77, 8, 4, 64, 192, [5, 0, 1000]),    # d = 64: four heads per tile
+    (1, 8192, 4, 2, 128, 128, [0]),          # 256 tiles: several per CTA, both accumulator buffers
+    (1, 300, 40, 8, 128, 5120, [4000]),      # 32B shapes (GQA 5:1)
+    (1, 256, 32, 32, 128, 4096, [0]),        # 7B shapes (MHA)
+])
+def test_qkv_proj_qknorm_rope_parity(B, T, H, G, d, D, offs):
+    x, w, gq, gk = qkv_inputs(B, T, H, G, d, D, 700 + T + D)
+    pos = torch.tensor(offs, dtype=torch.int32, device="cuda")
+    err = new_err()
+    got = L.qkv_proj_qknorm_rope(x, w, gq, gk, pos, H, G, d, err=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    check_qkv(got, x, w, gq, gk, offs, H, G, d, what=f"qkv {B}x{T} H{H} G{G} d{d} D{D}")
+
+
+def test_qkv_proj_yarn_and_workspace_reuse():
+    B, T, H, G, d, D = 2, 200, 4, 2, 128, 256
+    offs = [60000, 123]
+    x, w, gq, gk = qkv_inputs(B, T, H, G, d, D, 41)
+    pos = torch.tensor(offs, dtype=torch.int32, device="cuda")
+    ws = torch.full((L.qkv_proj_workspace_size(B * T),), 0x7f, dtype=torch.uint8, device="cuda")  # stale bytes
+    err = new_err()
+    a = L.qkv_proj_qknorm_rope(x, w, gq, gk, pos, H, G, d, factor=8.0, workspace=ws, err=err)
+    b = L.qkv_proj_qknorm_rope(x, w, gq, gk, pos, H, G, d, factor=8.0, workspace=ws, err=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    for u, v in zip(a, b):
+        assert torch.equal(u, v)
+    check_qkv(a, x, w, gq, gk, offs, H, G, d, yarn=8.0, what="qkv yarn")
+
+
+def test_qkv_proj_matches_unfused_path():
+    """The fused kernel against the GEMM + K1 pipeline it replaces, on the same inputs."""
+    B, T, H, G, d, D = 1, 384, 8, 2, 128, 512
+    x, w, gq, gk = qkv_inputs(B, T, H, G, d, D, 43)
+    pos = torch.tensor([17], dtype=torch.int32, device="cuda")
+    q, k, v = L.qkv_proj_qknorm_rope(x, w, gq, gk, pos, H, G, d)
+    y = (x.float().reshape(T, D) @ w.float().T).reshape(B, T, -1)
+    q2, k2, _ = L.qknorm_rope(y[..., :H * d].reshape(B, T, H, d).contiguous(),
+                              y[..., H * d:(H + G) * d].reshape(B, T, G, d).contiguous(), gq, gk, pos)
+    torch.cuda.synchronize()
+    # both round nearly equal f32 values to bf16 once: at most one bf16 ulp apart (2^-7 relative)
+    for a, b, n in [(q, q2, "q"), (k, k2, "k"), (v, y[..., (H + G) * d:].reshape(B, T, G, d), "v")]:
+        err = np.abs(f64(a) - f64(b))
+        assert (err <= 2.0 ** -7 * np.abs(f64(b)) + 1e-4).all(), f"fused vs unfused {n}: worst {err.max():.3e}"
+
+
+def test_qkv_proj_full_size_sampled_rows():
+    """7B at the prefill size (8192 tokens, D 4096, N 12288) and 32B at 2 x 8192."""
+    rng = np.random.default_rng(12)
+    for (B, T, H, G, D, seed) in [(1, 8192, 32, 32, 4096, 51), (2, 8192, 40, 8, 5120, 52)]:
+        d = 128
+        x = WL.randn_bf16((B, T, D), seed, "cuda")
+        w = (WL.randn_bf16(((H + 2 * G) * d, D), seed + 1, "cuda").float() / math.sqrt(D)).to(torch.bfloat16)
+        gq = torch.rand(H * d, device="cuda") + 0.5
+        gk = torch.rand(G * d, device="cuda") + 0.5
+        offs = [0] * B
+        pos = torch.tensor(offs, dtype=torch.int32, device="cuda")
+        err = new_err()
+        got = L.qkv_proj_qknorm_rope(x, w, gq, gk, pos, H, G, d, err=err)
+        torch.cuda.synchronize()
+        assert err.item() == 0
+        rows = sorted(set([(0, 0), (0, 127), (0, 128), (B - 1, T - 1)] +
+                          [(int(rng.integers(0, B)), int(rng.integers(0, T))) for _ in range(8)]))
+        check_qkv(got, x, w, gq, gk, offs, H, G, d, rows=rows, what=f"qkv full-size H{H}")
 
 
 # ---------------------------------------------------------------------------
