@@ -39,18 +39,57 @@ namespace olmo3 {
 
 constexpr int kBM = kPrefillBM;  // rows per query tile
 constexpr int kBN = kPrefillBN;  // keys per key tile
-constexpr int kRing = 4;
+#ifndef OLMO3_PF_RING
+#define OLMO3_PF_RING 4
+#endif
+#ifndef OLMO3_PF_QB_FAST
+#define OLMO3_PF_QB_FAST 0
+#endif
+constexpr int kRing = OLMO3_PF_RING;
 constexpr int kPfThreads = 384;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
+// Pairs q of a row's 64 score pairs with (q % kPolyDen) < kPolyNum take their
+// exponentials on the FMA pipe (exp2_poly2) instead of the transcendental unit.
+#ifndef OLMO3_PF_POLY_NUM
+#define OLMO3_PF_POLY_NUM 0
+#endif
+#ifndef OLMO3_PF_POLY_DEN
+#define OLMO3_PF_POLY_DEN 4
+#endif
+constexpr int kPolyNum = OLMO3_PF_POLY_NUM, kPolyDen = OLMO3_PF_POLY_DEN;
 #ifndef OLMO3_PF_CONTROL_REGS
-#define OLMO3_PF_CONTROL_REGS 64
+#define OLMO3_PF_CONTROL_REGS 72
 #endif
 // Register split between the control warpgroup and the two softmax warpgroups:
 // 128 x control + 256 x softmax must not exceed 384 x 168 (the launch budget).
 constexpr uint32_t kControlRegs = OLMO3_PF_CONTROL_REGS;
 constexpr uint32_t kSoftmaxRegs = ((384u * 168u - 128u * kControlRegs) / 256u) & ~7u;
 
+// 2^x for a pair of scores on the FMA and integer pipes, returned as f32 bit
+// patterns.  Range reduction x = j + f with j = round(x) (adding and removing
+// 1.5 * 2^23 leaves round(x) in the low mantissa bits of the sum) and |f| <= 1/2;
+// 2^f from a degree-3 polynomial fitted for minimum relative error on [-1/2, 1/2]
+// (max relative error 7.5e-5, far below the bf16 rounding of P); j is then added
+// to the exponent field.  x is clamped to >= -126 first (so the exponent field
+// stays >= 0): a masked score (-inf) gives a value below 2^-126, nothing next to
+// the 2^0 of the row maximum, and while a row has seen no unmasked score its sum
+// is cleared by the first rescale (alpha = 2^-inf = 0).
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, uint32_t &b0, uint32_t &b1) {
+  const uint64_t magic = f2pack(12582912.0f, 12582912.0f), neg_one = f2pack(-1.0f, -1.0f);
+  const uint64_t c0 = f2pack(0.99992812f, 0.99992812f), c1 = f2pack(0.69326097f, 0.69326097f);
+  const uint64_t c2 = f2pack(0.24261054f, 0.24261054f), c3 = f2pack(0.055171322f, 0.055171322f);
+  const uint64_t x = f2pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+  const uint64_t t = fadd2(x, magic);
+  const uint64_t j = ffma2(magic, neg_one, t);   // round(x), exactly
+  const uint64_t fr = ffma2(j, neg_one, x);      // x - round(x)
+  const uint64_t p = ffma2(ffma2(ffma2(c3, fr, c2), fr, c1), fr, c0);
+  float p0, p1, t0, t1;
+  f2unpack(p, p0, p1);
+  f2unpack(t, t0, t1);
+  b0 = __float_as_uint(p0) + (__float_as_uint(t0) << 23);
+  b1 = __float_as_uint(p1) + (__float_as_uint(t1) << 23);
+}
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -116,8 +155,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint8_t *sQ = smem + LY::kOffQ;
   uint8_t *sRing = smem + LY::kOffRing;
 
+#if OLMO3_PF_QB_FAST
+  const int h = blockIdx.y;
+  const int qb = n_blocks - 1 - static_cast<int>(blockIdx.x);  // longest rows first
+#else
   const int h = blockIdx.x;
   const int qb = n_blocks - 1 - static_cast<int>(blockIdx.y);  // longest rows first
+#endif
   const int b = blockIdx.z;
   const int g = h / (H / G);
   const int q0 = qb * 2 * kBM;
@@ -227,35 +271,35 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int i = max(0, issued - kRing); i < issued; ++i)
           mbar_wait(&ring_full[i % kRing], (i / kRing) & 1, nullptr);
       }
-    } else if (warp == 9 && lane == 0) {
+    } else if (warp == 9) {
       // ------------------------------ MMA issuer ------------------------------
+      // The whole warp runs this loop with the same values (descriptors stay in
+      // uniform registers); one elected lane issues each MMA and commit.
       const uint32_t aQ = smem_u32(sQ), aR = smem_u32(sRing);
       int cnt_pv[2] = {0, 0};
-      bool ok = mbar_wait(&q_full, 0, &s_abort);
+      bool ok = mbar_wait_warp(&q_full, 0, &s_abort);
       auto item_ready = [&](int i) -> bool {
-        return mbar_wait(&ring_full[i % kRing], (i / kRing) & 1, &s_abort);
+        return mbar_wait_warp(&ring_full[i % kRing], (i / kRing) & 1, &s_abort);
       };
       auto issue_s = [&](int w, int j) {  // S_w = Q_w K_j^T (K_j is item 2j)
-        const uint32_t kb = aR + ((2 * j) % kRing) * LY::kKVBytes;
-        const uint32_t qw = aQ + w * LY::kQBytes;
+        const uint64_t dq = sw128_desc(aQ + w * LY::kQBytes, 16, 1024);
+        const uint64_t dk = sw128_desc(aR + ((2 * j) % kRing) * LY::kKVBytes, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
-          umma_bf16(tmem + w * kBN, sw128_desc(qw + off, 16, 1024), sw128_desc(kb + off, 16, 1024), IDESC_S,
-                    kk > 0);
+          const uint32_t off16 = ((kk >> 2) * (kBN * 128) + (kk & 3) * 32) >> 4;  // address field, 16-byte units
+          umma_bf16_elect(tmem + w * kBN, dq + off16, dk + off16, IDESC_S, kk > 0);
         }
-        umma_commit(&s_full[w]);
+        umma_commit_elect(&s_full[w]);
       };
       auto issue_pv = [&](int w, int j) -> bool {  // O_w += P_w V_j (V_j is item 2j+1, P_w in TMEM)
-        if (!mbar_wait(&p_full[w], cnt_pv[w] & 1, &s_abort)) return false;
+        if (!mbar_wait_warp(&p_full[w], cnt_pv[w] & 1, &s_abort)) return false;
         tc_fence_after();
-        const uint32_t vb = aR + ((2 * j + 1) % kRing) * LY::kKVBytes;
+        const uint64_t dv = sw128_desc(aR + ((2 * j + 1) % kRing) * LY::kKVBytes, kBN * 128, 1024);
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          umma_bf16_ts(tmem + 256 + w * D, tmem + w * kBN + kk * 8, sw128_desc(vb + kk * (16 * 128), kBN * 128, 1024),
-                       IDESC_O, (cnt_pv[w] > 0 || kk > 0));
-        }
-        umma_commit(&o_done[w]);
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          umma_bf16_ts_elect(tmem + 256 + w * D, tmem + w * kBN + kk * 8, dv + kk * ((16 * 128) >> 4), IDESC_O,
+                             (cnt_pv[w] > 0 || kk > 0));
+        umma_commit_elect(&o_done[w]);
         ++cnt_pv[w];
         return true;
       };
@@ -267,7 +311,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tc_fence_after();
         if (active(0, 0)) issue_s(0, 0);
         if (active(1, 0)) issue_s(1, 0);
-        umma_commit(&ring_empty[0]);
+        umma_commit_elect(&ring_empty[0]);
       }
       for (int j = 0; ok && j < n_kt; ++j) {
         if (!(ok = item_ready(2 * j + 1))) break;  // V_j
@@ -280,18 +324,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           if (active(0, j + 1)) issue_s(0, j + 1);
         }
         if (active(1, j) && !(ok = issue_pv(1, j))) break;
-        umma_commit(&ring_empty[(2 * j + 1) % kRing]);  // V_j consumed by both PVs
+        umma_commit_elect(&ring_empty[(2 * j + 1) % kRing]);  // V_j consumed by both PVs
         if (more) {
           if (active(1, j + 1)) issue_s(1, j + 1);
-          umma_commit(&ring_empty[(2 * j + 2) % kRing]);  // K_{j+1} consumed by both S
+          umma_commit_elect(&ring_empty[(2 * j + 2) % kRing]);  // K_{j+1} consumed by both S
         }
       }
-      if (!ok) {
+      if (!ok && lane == 0) {
         s_abort = 1;
         set_dev_error(err, OLMO3_DEVERR_TIMEOUT);
       }
-      umma_commit(&mma_drain);  // every MMA issued has completed before tensor memory is freed
-      mbar_wait(&mma_drain, 0, nullptr);
+      umma_commit_elect(&mma_drain);  // every MMA issued has completed before tensor memory is freed
+      mbar_wait_warp(&mma_drain, 0, nullptr);
     }
   } else {
     regs_inc<kSoftmaxRegs>();
@@ -366,8 +410,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         f2unpack(ffma2(f2pack(__uint_as_float(sr[q >> 4][(2 * q) & 31]), __uint_as_float(sr[q >> 4][(2 * q + 1) & 31])),
                        scale2, negm2),
                  x0, x1);
-        const uint32_t b0 = __float_as_uint(ex2(x0));
-        const uint32_t b1 = __float_as_uint(ex2(x1));
+        uint32_t b0, b1;
+        if (kPolyNum > 0 && (q % kPolyDen) < kPolyNum) {
+          exp2_poly2(x0, x1, b0, b1);
+        } else {
+          b0 = __float_as_uint(ex2(x0));
+          b1 = __float_as_uint(ex2(x1));
+        }
         pk[q] = __byte_perm(b0, b1, 0x7632);
         sm2[q & 3] = fadd2(sm2[q & 3], f2pack(__uint_as_float(b0 & 0xFFFF0000u), __uint_as_float(b1 & 0xFFFF0000u)));
       }
@@ -452,7 +501,11 @@ static cudaError_t launch_pf(const CUtensorMap &tmQ, const CUtensorMap &tmK, con
     attr_set = true;
   }
   const int n_blocks = (Tq + 2 * kBM - 1) / (2 * kBM);
+#if OLMO3_PF_QB_FAST
+  dim3 grid(n_blocks, H, B);
+#else
   dim3 grid(H, n_blocks, B);
+#endif
   attn_prefill_kernel<D, MODE><<<grid, kPfThreads, LY::kDynBytes, stream>>>(
       tmQ, tmK, tmV, static_cast<__nv_bfloat16 *>(out), lse_out, Tq, Tk, H, G, layer_type, window,
       scale * 1.4426950408889634f, n_blocks, pos_offset, seq_base, err);

@@ -387,40 +387,40 @@ __global__ void __launch_bounds__(kPThreads, 1)
     }
   } else if (warp == 5) {
     // ------------------------------ MMA issuer --------------------------------
-    if (lane == 0) {
-      int it = 0, lt = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++lt) {
-        const int buf = lt & 1;
-        if (lt >= 2 && !mbar_wait(&acc_empty[buf], ((lt >> 1) & 1) ^ 1, &s_abort)) {
+    // The whole warp runs the loop with the same values (descriptors stay in
+    // uniform registers); one elected lane issues each MMA and commit.
+    int it = 0, lt = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++lt) {
+      const int buf = lt & 1;
+      if (lt >= 2 && !mbar_wait_warp(&acc_empty[buf], ((lt >> 1) & 1) ^ 1, &s_abort)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t acc = tmem + buf * kPBN;
+      for (int kc = 0; kc < nk; ++kc, ++it) {
+        const int st = it % kPStages;
+        if (!mbar_wait_warp(&full_bar[st], (it / kPStages) & 1, &s_abort)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t acc = tmem + buf * kPBN;
-        for (int kc = 0; kc < nk; ++kc, ++it) {
-          const int st = it % kPStages;
-          if (!mbar_wait(&full_bar[st], (it / kPStages) & 1, &s_abort)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t sa = smem_u32(smem + st * kPStageBytes), sb = sa + kPABytes;
+        const uint32_t sa = smem_u32(smem + st * kPStageBytes);
+        const uint64_t da = sw128_desc(sa, 16, 1024), db = sw128_desc(sa + kPABytes, 16, 1024);
 #pragma unroll
-          for (int kk = 0; kk < kPBK / 16; ++kk)
-            umma_bf16(acc, sw128_desc(sa + kk * 32, 16, 1024), sw128_desc(sb + kk * 32, 16, 1024), IDESC,
-                      (kc > 0 || kk > 0));
-          umma_commit(&empty_bar[st]);
-        }
-        if (ok) umma_commit(&acc_full[buf]);
+        for (int kk = 0; kk < kPBK / 16; ++kk)
+          umma_bf16_elect(acc, da + kk * 2, db + kk * 2, IDESC, (kc > 0 || kk > 0));  // +32 bytes per K step
+        umma_commit_elect(&empty_bar[st]);
       }
-      if (!ok) {
-        if (!s_abort) set_dev_error(err, OLMO3_DEVERR_TIMEOUT);
-        s_abort = 1;
-      }
-      umma_commit(&drain_bar);  // completes once every MMA issued above has
-      mbar_wait(&drain_bar, 0, nullptr);
+      if (ok) umma_commit_elect(&acc_full[buf]);
     }
+    if (!ok && lane == 0) {
+      if (!s_abort) set_dev_error(err, OLMO3_DEVERR_TIMEOUT);
+      s_abort = 1;
+    }
+    umma_commit_elect(&drain_bar);  // completes once every MMA issued above has
+    mbar_wait_warp(&drain_bar, 0, nullptr);
   } else {
     // ------------------------------ epilogue ----------------------------------
     int lt = 0;
