@@ -15,7 +15,8 @@
 //   WG1 (warps 4-7)  the same for tile B.
 //   WG2 warp 8       TMA producer: both Q tiles once, then K_j, V_j, K_j+1, ... into
 //                    a 4-slot ring (each slot holds one 128-key K or V tile).
-//       warp 9       TMEM allocator and MMA issuer (one thread).
+//       warp 9       TMEM allocator and MMA issuer (the whole warp runs the issue
+//                    loop on warp-uniform values; one elected lane issues).
 // WG2 gives registers to the softmax warpgroups (setmaxnreg).
 // Tensor memory (512 columns): S_A [0,128), S_B [128,256) fp32 score tiles,
 // O_A [256, 256+d), O_B [256+d, 256+2d) fp32 accumulators.  P (bf16, two per
@@ -25,7 +26,9 @@
 // at 128 rows x 128 columns, which is what the shared-memory bandwidth allows).
 // Tensor-core order per key tile j:  PV_A(j), S_A(j+1), PV_B(j), S_B(j+1): while
 // one softmax warpgroup turns its S into P the tensor core works for the other
-// tile, so the two warpgroups alternate against a busy tensor core.  A row's running max is only
+// tile, so the two warpgroups alternate against a busy tensor core.  P is handed
+// over in two halves of 64 keys (two barriers), so the first half of PV starts
+// while the softmax computes the second.  A row's running max is only
 // raised (and O rescaled in TMEM) when it grows by more than 2^8, so P <= 256 and
 // most tiles skip the rescale.
 // Every wait is bounded: on a timeout the CTA records OLMO3_DEVERR_TIMEOUT,
@@ -39,25 +42,11 @@ namespace olmo3 {
 
 constexpr int kBM = kPrefillBM;  // rows per query tile
 constexpr int kBN = kPrefillBN;  // keys per key tile
-#ifndef OLMO3_PF_RING
-#define OLMO3_PF_RING 4
-#endif
-#ifndef OLMO3_PF_QB_FAST
-#define OLMO3_PF_QB_FAST 0
-#endif
-constexpr int kRing = OLMO3_PF_RING;
+constexpr int kRing = 4;
 constexpr int kPfThreads = 384;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
-// Pairs q of a row's 64 score pairs with (q % kPolyDen) < kPolyNum take their
-// exponentials on the FMA pipe (exp2_poly2) instead of the transcendental unit.
-#ifndef OLMO3_PF_POLY_NUM
-#define OLMO3_PF_POLY_NUM 0
-#endif
-#ifndef OLMO3_PF_POLY_DEN
-#define OLMO3_PF_POLY_DEN 4
-#endif
-constexpr int kPolyNum = OLMO3_PF_POLY_NUM, kPolyDen = OLMO3_PF_POLY_DEN;
+
 #ifndef OLMO3_PF_CONTROL_REGS
 #define OLMO3_PF_CONTROL_REGS 72
 #endif
@@ -66,30 +55,6 @@ constexpr int kPolyNum = OLMO3_PF_POLY_NUM, kPolyDen = OLMO3_PF_POLY_DEN;
 constexpr uint32_t kControlRegs = OLMO3_PF_CONTROL_REGS;
 constexpr uint32_t kSoftmaxRegs = ((384u * 168u - 128u * kControlRegs) / 256u) & ~7u;
 
-// 2^x for a pair of scores on the FMA and integer pipes, returned as f32 bit
-// patterns.  Range reduction x = j + f with j = round(x) (adding and removing
-// 1.5 * 2^23 leaves round(x) in the low mantissa bits of the sum) and |f| <= 1/2;
-// 2^f from a degree-3 polynomial fitted for minimum relative error on [-1/2, 1/2]
-// (max relative error 7.5e-5, far below the bf16 rounding of P); j is then added
-// to the exponent field.  x is clamped to >= -126 first (so the exponent field
-// stays >= 0): a masked score (-inf) gives a value below 2^-126, nothing next to
-// the 2^0 of the row maximum, and while a row has seen no unmasked score its sum
-// is cleared by the first rescale (alpha = 2^-inf = 0).
-__device__ __forceinline__ void exp2_poly2(float x0, float x1, uint32_t &b0, uint32_t &b1) {
-  const uint64_t magic = f2pack(12582912.0f, 12582912.0f), neg_one = f2pack(-1.0f, -1.0f);
-  const uint64_t c0 = f2pack(0.99992812f, 0.99992812f), c1 = f2pack(0.69326097f, 0.69326097f);
-  const uint64_t c2 = f2pack(0.24261054f, 0.24261054f), c3 = f2pack(0.055171322f, 0.055171322f);
-  const uint64_t x = f2pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
-  const uint64_t t = fadd2(x, magic);
-  const uint64_t j = ffma2(magic, neg_one, t);   // round(x), exactly
-  const uint64_t fr = ffma2(j, neg_one, x);      // x - round(x)
-  const uint64_t p = ffma2(ffma2(ffma2(c3, fr, c2), fr, c1), fr, c0);
-  float p0, p1, t0, t1;
-  f2unpack(p, p0, p1);
-  f2unpack(t, t0, t1);
-  b0 = __float_as_uint(p0) + (__float_as_uint(t0) << 23);
-  b1 = __float_as_uint(p1) + (__float_as_uint(t1) << 23);
-}
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -147,7 +112,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t q_full, ring_full[kRing], ring_empty[kRing];
-  __shared__ uint64_t s_full[2], p_full[2], o_done[2], mma_drain;
+  __shared__ uint64_t s_full[2], p_full[2][2], o_done[2], mma_drain;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
 
@@ -155,13 +120,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint8_t *sQ = smem + LY::kOffQ;
   uint8_t *sRing = smem + LY::kOffRing;
 
-#if OLMO3_PF_QB_FAST
-  const int h = blockIdx.y;
-  const int qb = n_blocks - 1 - static_cast<int>(blockIdx.x);  // longest rows first
-#else
   const int h = blockIdx.x;
   const int qb = n_blocks - 1 - static_cast<int>(blockIdx.y);  // longest rows first
-#endif
   const int b = blockIdx.z;
   const int g = h / (H / G);
   const int q0 = qb * 2 * kBM;
@@ -219,7 +179,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(&s_full[w], 1);
-      mbar_init(&p_full[w], kBM);
+      mbar_init(&p_full[w][0], kBM);
+      mbar_init(&p_full[w][1], kBM);
       mbar_init(&o_done[w], 1);
     }
     mbar_init(&mma_drain, 1);
@@ -292,13 +253,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         umma_commit_elect(&s_full[w]);
       };
       auto issue_pv = [&](int w, int j) -> bool {  // O_w += P_w V_j (V_j is item 2j+1, P_w in TMEM)
-        if (!mbar_wait_warp(&p_full[w], cnt_pv[w] & 1, &s_abort)) return false;
-        tc_fence_after();
         const uint64_t dv = sw128_desc(aR + ((2 * j + 1) % kRing) * LY::kKVBytes, kBN * 128, 1024);
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          umma_bf16_ts_elect(tmem + 256 + w * D, tmem + w * kBN + kk * 8, dv + kk * ((16 * 128) >> 4), IDESC_O,
-                             (cnt_pv[w] > 0 || kk > 0));
+        for (int half = 0; half < 2; ++half) {  // keys [64 half, 64 half + 64): P columns [32 half, +32)
+          if (!mbar_wait_warp(&p_full[w][half], cnt_pv[w] & 1, &s_abort)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int k4 = 0; k4 < kBN / 32; ++k4) {
+            const int kk = half * (kBN / 32) + k4;
+            umma_bf16_ts_elect(tmem + 256 + w * D, tmem + w * kBN + kk * 8, dv + kk * ((16 * 128) >> 4), IDESC_O,
+                               (cnt_pv[w] > 0 || kk > 0));
+          }
+        }
         umma_commit_elect(&o_done[w]);
         ++cnt_pv[w];
         return true;
@@ -399,34 +365,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
       const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
       const uint64_t negm2 = f2pack(neg_m, neg_m);
-      // P = 2^(s*scale - m), truncated to bf16 (the upper 16 bits, packed two per
-      // column); the row sum adds the same truncated values, so the normalisation
-      // matches what the tensor core multiplies.
-      uint64_t sm2[4] = {0, 0, 0, 0};
-      uint32_t pk[kBN / 2];
-#pragma unroll
-      for (int q = 0; q < kBN / 2; ++q) {
-        float x0, x1;
-        f2unpack(ffma2(f2pack(__uint_as_float(sr[q >> 4][(2 * q) & 31]), __uint_as_float(sr[q >> 4][(2 * q + 1) & 31])),
-                       scale2, negm2),
-                 x0, x1);
-        uint32_t b0, b1;
-        if (kPolyNum > 0 && (q % kPolyDen) < kPolyNum) {
-          exp2_poly2(x0, x1, b0, b1);
-        } else {
-          b0 = __float_as_uint(ex2(x0));
-          b1 = __float_as_uint(ex2(x1));
-        }
-        pk[q] = __byte_perm(b0, b1, 0x7632);
-        sm2[q & 3] = fadd2(sm2[q & 3], f2pack(__uint_as_float(b0 & 0xFFFF0000u), __uint_as_float(b1 & 0xFFFF0000u)));
-      }
-      float s0, s1, s2, s3, s4, s5, s6, s7;
-      f2unpack(sm2[0], s0, s1);
-      f2unpack(sm2[1], s2, s3);
-      f2unpack(sm2[2], s4, s5);
-      f2unpack(sm2[3], s6, s7);
-      lsum = lsum * alpha + (((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7)));
-
+      // O_w holds PV_w(j-1) (complete: see above); rescale it before PV_w(j) adds to it.
       if (cnt > 0 && __any_sync(0xffffffffu, resc)) {
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
@@ -438,12 +377,38 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           tmem_st32(tO + c * 32, orr);
         }
       }
-      // P_w(j) -> the first 64 columns of S_w
-      tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&p_full[w]);
+      // P = 2^(s*scale - m), truncated to bf16 (the upper 16 bits, packed two per
+      // column); the row sum adds the same truncated values, so the normalisation
+      // matches what the tensor core multiplies.  P goes to the first 64 columns of
+      // S_w in two halves of 64 keys, each announced on its own barrier, so the
+      // tensor core starts on the first half while the second is computed.
+      uint64_t sm2[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[kBN / 4];
+#pragma unroll
+        for (int qq = 0; qq < kBN / 4; ++qq) {
+          const int q = half * (kBN / 4) + qq;
+          float x0, x1;
+          f2unpack(ffma2(f2pack(__uint_as_float(sr[q >> 4][(2 * q) & 31]), __uint_as_float(sr[q >> 4][(2 * q + 1) & 31])),
+                         scale2, negm2),
+                   x0, x1);
+          const uint32_t b0 = __float_as_uint(ex2(x0));
+          const uint32_t b1 = __float_as_uint(ex2(x1));
+          pk[qq] = __byte_perm(b0, b1, 0x7632);
+          sm2[q & 3] = fadd2(sm2[q & 3], f2pack(__uint_as_float(b0 & 0xFFFF0000u), __uint_as_float(b1 & 0xFFFF0000u)));
+        }
+        tmem_st32(tS + half * 32, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full[w][half]);
+      }
+      float s0, s1, s2, s3, s4, s5, s6, s7;
+      f2unpack(sm2[0], s0, s1);
+      f2unpack(sm2[1], s2, s3);
+      f2unpack(sm2[2], s4, s5);
+      f2unpack(sm2[3], s6, s7);
+      lsum = lsum * alpha + (((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7)));
     }
     if (ok && cnt > 0) ok = __all_sync(0xffffffffu, mbar_wait(&o_done[w], (cnt - 1) & 1, &s_abort));
     if (!ok) {
@@ -501,11 +466,7 @@ static cudaError_t launch_pf(const CUtensorMap &tmQ, const CUtensorMap &tmK, con
     attr_set = true;
   }
   const int n_blocks = (Tq + 2 * kBM - 1) / (2 * kBM);
-#if OLMO3_PF_QB_FAST
-  dim3 grid(n_blocks, H, B);
-#else
   dim3 grid(H, n_blocks, B);
-#endif
   attn_prefill_kernel<D, MODE><<<grid, kPfThreads, LY::kDynBytes, stream>>>(
       tmQ, tmK, tmV, static_cast<__nv_bfloat16 *>(out), lse_out, Tq, Tk, H, G, layer_type, window,
       scale * 1.4426950408889634f, n_blocks, pos_offset, seq_base, err);
