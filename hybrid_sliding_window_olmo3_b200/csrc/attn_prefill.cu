@@ -30,7 +30,8 @@
 // over in two halves of 64 keys (two barriers), so the first half of PV starts
 // while the softmax computes the second.  A row's running max is only
 // raised (and O rescaled in TMEM) when it grows by more than 2^8, so P <= 256 and
-// most tiles skip the rescale.
+// most tiles skip the rescale.  P is rounded to nearest bf16 for the PV product;
+// the row sum adds the f32 weights.
 // Every wait is bounded: on a timeout the CTA records OLMO3_DEVERR_TIMEOUT,
 // drains its copies and MMAs in flight, frees its tensor memory and exits.
 #include <math.h>
@@ -377,11 +378,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           tmem_st32(tO + c * 32, orr);
         }
       }
-      // P = 2^(s*scale - m), truncated to bf16 (the upper 16 bits, packed two per
-      // column); the row sum adds the same truncated values, so the normalisation
-      // matches what the tensor core multiplies.  P goes to the first 64 columns of
-      // S_w in two halves of 64 keys, each announced on its own barrier, so the
-      // tensor core starts on the first half while the second is computed.
+      // P = 2^(s*scale - m), rounded to nearest bf16 (packed two per column) for the
+      // tensor core; the row sum adds the f32 values.  P goes to the first 64
+      // columns of S_w in two halves of 64 keys, each announced on its own barrier,
+      // so the tensor core starts on the first half while the second is computed.
       uint64_t sm2[4] = {0, 0, 0, 0};
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
@@ -393,10 +393,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           f2unpack(ffma2(f2pack(__uint_as_float(sr[q >> 4][(2 * q) & 31]), __uint_as_float(sr[q >> 4][(2 * q + 1) & 31])),
                          scale2, negm2),
                    x0, x1);
-          const uint32_t b0 = __float_as_uint(ex2(x0));
-          const uint32_t b1 = __float_as_uint(ex2(x1));
-          pk[qq] = __byte_perm(b0, b1, 0x7632);
-          sm2[q & 3] = fadd2(sm2[q & 3], f2pack(__uint_as_float(b0 & 0xFFFF0000u), __uint_as_float(b1 & 0xFFFF0000u)));
+          const float e0 = ex2(x0), e1 = ex2(x1);
+          pk[qq] = f2_to_bf2(e0, e1);
+          sm2[q & 3] = fadd2(sm2[q & 3], f2pack(e0, e1));
         }
         tmem_st32(tS + half * 32, pk);
         tmem_wait_st();

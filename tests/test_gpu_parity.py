@@ -3,10 +3,10 @@ fp64 oracle on the same seeded inputs.
 
 Bars: masks, layer types, cache slots and cache contents bit-exact; QK-norm +
 RoPE within bf16 rounding (|err| <= 2^-8 |ref| + 1e-4); attention outputs
-max-abs <= 2e-2 and mean-abs <= 2e-3.  LSE: the prefill kernel rounds each
-softmax weight P toward zero to bf16 (relative error below 2^-7) and its row sum
-adds those same rounded weights, so its log-sum-exp is below the exact one by at
-most ln(1 / (1 - 2^-7)) = 0.0079 (plus fp32 rounding); the bar is 1e-2.
+max-abs <= 2e-2 and mean-abs <= 2e-3.  LSE: every attention kernel adds the
+f32 softmax weights (only the copy of P that feeds the bf16 product is rounded),
+so the log-sum-exp carries f32 and ex2.approx rounding only (relative ~1e-6 on
+sums of up to 65,536 terms, a few 1e-6 absolute); the bar is 1e-3.
 """
 import math
 
@@ -22,7 +22,7 @@ from hybrid_sliding_window_olmo3_b200 import workloads as WL
 pytestmark = pytest.mark.gpu
 
 TYP = {L.SLIDING: O.SLIDING, L.FULL: O.FULL}
-MAX_ABS, MEAN_ABS, LSE_ABS = 2e-2, 2e-3, 1e-2
+MAX_ABS, MEAN_ABS, LSE_ABS = 2e-2, 2e-3, 1e-3
 
 
 @pytest.fixture(scope="module", autouse=True)

@@ -418,6 +418,23 @@ def test_qkv_projection_with_identity_weights_is_qknorm_rope_of_the_input():
     np.testing.assert_allclose(v, x[..., (H + G) * d:].reshape(B, T, G, d), atol=0)
 
 
+def test_qkv_projection_with_explicit_plain_frequencies_matches_the_default_path():
+    rng = np.random.default_rng(16)
+    B, T, H, G, d, D = 1, 5, 2, 1, 8, 12
+    x, w = rng.standard_normal((B, T, D)), rng.standard_normal(((H + 2 * G) * d, D))
+    gq, gk = rng.uniform(0.5, 1.5, H * d), rng.uniform(0.5, 1.5, G * d)
+    pos = np.arange(7, 7 + T)[None]
+    a = O.qkv_projection(x, w, gq, gk, pos, H, G, d)
+    b = O.qkv_projection(x, w, gq, gk, pos, H, G, d, inv_freq=O.rope_inv_freq(d, 500000.0), out_scale=1.0)
+    for u, v in zip(a, b):
+        np.testing.assert_allclose(u, v, atol=1e-12)
+    # a YaRN temperature multiplies the rotated q and k, and leaves v alone
+    c = O.qkv_projection(x, w, gq, gk, pos, H, G, d, inv_freq=O.rope_inv_freq(d, 500000.0), out_scale=1.25)
+    np.testing.assert_allclose(c[0], 1.25 * a[0], atol=1e-12)
+    np.testing.assert_allclose(c[1], 1.25 * a[1], atol=1e-12)
+    np.testing.assert_array_equal(c[2], a[2])
+
+
 def test_kv_sizing_matches_the_pages():
     g = {r[0]: float(r[1]) for r in read_golden("kv_sizing.txt")}
     t32 = O.layer_types(32)
