@@ -27,10 +27,11 @@
 // CTA's next tile run while its epilogue waits.
 //
 // Tile order.  Output columns are split into phases (QKV: the q columns, then the k
-// and v columns; Wo: one phase), and each phase runs its row blocks in order, all of
-// the phase's column tiles of a row block back to back.  A phase's weights (32-64 MB
-// for the 7B and 32B models) then stay in L2 while every row block streams past
-// them, instead of the whole W_qkv cycling through L2 once per wave.
+// and v columns, as one phase or, when their weights exceed 48 MB, as two; Wo: one
+// phase), and each phase runs its row blocks in order, all of the phase's column
+// tiles of a row block back to back.  A phase's weights (10-52 MB for the 7B and 32B
+// models) then stay in L2 while every row block streams past them, instead of the
+// whole W_qkv cycling through L2 once per wave.
 // Deadlock freedom: position p of this order runs on CTA p mod grid after the tile at
 // p - grid.  A tile waits only for the tiles of its norm group (its row block's q
 // tiles, or k tiles, or all Wo tiles), which sit within fewer than `grid` consecutive
@@ -55,6 +56,8 @@ constexpr int kPABytes = kPBM * kPBK * 2;
 constexpr int kPBBytes = kPBN * kPBK * 2;
 constexpr int kPStageBytes = kPABytes + kPBBytes;
 constexpr int kPSmemBytes = kPStages * kPStageBytes + 1024;
+// Weights of one QKV column phase above this size get a phase each for k and v.
+constexpr size_t kQkvPhaseBytes = static_cast<size_t>(48) << 20;
 
 // QKV epilogue: columns [0, Hd) of Y are q, [Hd, Hd + Gd) k, the rest v.
 template <int D>
@@ -545,9 +548,12 @@ cudaError_t launch_qkv_proj(const CUtensorMap &tmX, const CUtensorMap &tmW, void
   int *abort_flag = count + 2 * rb;
   const size_t zero_bytes = proj_gemm_flags_bytes(M, 2);
   const int N = (H + 2 * G) * d;
-  // phases: the q columns, then the k and v columns
-  const int phase_cols[2] = {H * d / kPBN, 2 * G * d / kPBN};
-  const TileOrder order = make_order(M, phase_cols, 2);
+  // phases: the q columns, then the k and v columns, as one phase when their
+  // weights are small enough to stay in L2 next to the streamed rows, else two
+  const size_t kv_weight_bytes = static_cast<size_t>(2 * G * d) * Dm * 2;
+  const bool split_kv = kv_weight_bytes > kQkvPhaseBytes;
+  const int phase_cols[3] = {H * d / kPBN, (split_kv ? 1 : 2) * G * d / kPBN, G * d / kPBN};
+  const TileOrder order = make_order(M, phase_cols, split_kv ? 3 : 2);
   const int group = (H * d > G * d ? H * d : G * d) / kPBN;
   if (d == 64) {
     QkvEpilogue<64> ep{static_cast<__nv_bfloat16 *>(q), static_cast<__nv_bfloat16 *>(k),

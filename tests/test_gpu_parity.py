@@ -443,6 +443,29 @@ def test_chunked_prefill_equals_one_shot(typ):
     assert p0 == Ttot
 
 
+@pytest.mark.parametrize("B,H,G", [(1, 32, 32), (2, 40, 8)])
+def test_chunked_prefill_full_size_sampled_rows(B, H, G):
+    """The bench's chunked workloads: T = 8192 in four chunks of 2048 through a window-sized
+    ring (sliding) or a linear cache (full), checked on sampled rows of every chunk."""
+    rng = np.random.default_rng(3 + B)
+    T, d, W, C = 8192, 128, 4096, 2048
+    rows = sorted(set([0, 2047, 2048, 2049, 4095, 4096, 6143, 6144, 8191] + rng.integers(0, T, 6).tolist()))
+    for typ in (L.SLIDING, L.FULL):
+        q, k, v, _, _ = WL.qkv_bf16(B, T, H, G, d, 20261206, layer=typ)
+        tq, tk, tv = q.cuda(), k.cuda(), v.cuda()
+        cache = L.KVCache(typ, B, G, d, W, capacity=W if typ == L.SLIDING else T)
+        out = torch.empty_like(tq)
+        err = new_err()
+        for p0 in range(0, T, C):
+            pos = torch.full((B,), p0, dtype=torch.int32, device="cuda")
+            out[:, p0:p0 + C] = L.attn_prefill_chunk(tq[:, p0:p0 + C].contiguous(), tk[:, p0:p0 + C].contiguous(),
+                                                     tv[:, p0:p0 + C].contiguous(), cache, pos, err=err)
+        torch.cuda.synchronize()
+        assert err.item() == 0
+        ro, _ = O.prefill_attention(f64(q), f64(k), f64(v), TYP[typ], W, rows=rows)
+        close_attn(f64(out[:, rows]), ro, f"chunked full size type {typ}")
+
+
 # ---------------------------------------------------------------------------
 # Output side: projection + reordered post-norm + residual (tcgen05 GEMM)
 # ---------------------------------------------------------------------------
