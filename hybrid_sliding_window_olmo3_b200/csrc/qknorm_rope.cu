@@ -9,9 +9,11 @@
 //
 // Memory-bound: every byte of q and k is read once and written once.  Each
 // thread owns "pair chunks" (8 features i..i+7 of a head and their rotation
-// partners i+d/2..i+d/2+7), loads them with 16-byte vector loads, keeps them in
-// registers across the block reduction of the sum of squares, and rotates with
-// cos/sin that 64 threads form in fp64 once per token.
+// partners i+d/2..i+d/2+7), loads them with 16-byte vector loads and keeps them in
+// registers across the block reduction of the sum of squares (bf16 inputs stay
+// packed, 4 registers per chunk, so that enough CTAs fit on an SM to keep HBM
+// busy).  64 threads form cos/sin once per token: the angle is reduced to
+// [-pi, pi] in fp64, then evaluated in fp32.
 #include "common.cuh"
 #include "internal.h"
 
@@ -55,10 +57,36 @@ __device__ __forceinline__ float block_sum(float v, float *red) {
   return s;
 }
 
-// Loads the pair chunks of one row (n_heads heads) owned by this thread.
+// Register copy of one pair chunk: packed bf16 (uint4) or 8 floats.
+template <typename Tin> struct Chunk;
+template <> struct Chunk<__nv_bfloat16> {
+  uint4 u;
+  __device__ __forceinline__ void load(const __nv_bfloat16 *p) { u = *reinterpret_cast<const uint4 *>(p); }
+  __device__ __forceinline__ void get(float (&x)[8]) const {
+    float2 f;
+    f = bf2_to_f2(u.x); x[0] = f.x; x[1] = f.y;
+    f = bf2_to_f2(u.y); x[2] = f.x; x[3] = f.y;
+    f = bf2_to_f2(u.z); x[4] = f.x; x[5] = f.y;
+    f = bf2_to_f2(u.w); x[6] = f.x; x[7] = f.y;
+  }
+};
+template <> struct Chunk<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float *p) {
+    a = reinterpret_cast<const float4 *>(p)[0];
+    b = reinterpret_cast<const float4 *>(p)[1];
+  }
+  __device__ __forceinline__ void get(float (&x)[8]) const {
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  }
+};
+
+// Loads the pair chunks of one row (n_heads heads) owned by this thread and
+// returns their sum of squares.
 template <typename Tin, int D>
-__device__ __forceinline__ float load_row(const Tin *row, int n_heads, float (&lo)[kMaxChunks][8],
-                                          float (&hi)[kMaxChunks][8]) {
+__device__ __forceinline__ float load_row(const Tin *row, int n_heads, Chunk<Tin> (&lo)[kMaxChunks],
+                                          Chunk<Tin> (&hi)[kMaxChunks]) {
   constexpr int CPH = D / 16;  // pair chunks per head
   float ssq = 0.f;
 #pragma unroll
@@ -66,32 +94,38 @@ __device__ __forceinline__ float load_row(const Tin *row, int n_heads, float (&l
     const int ci = threadIdx.x + c * kNormThreads;
     if (ci < n_heads * CPH) {
       const int h = ci / CPH, i0 = (ci % CPH) * 8;
-      load8(row + h * D + i0, lo[c]);
-      load8(row + h * D + D / 2 + i0, hi[c]);
+      lo[c].load(row + h * D + i0);
+      hi[c].load(row + h * D + D / 2 + i0);
+      float a[8], b[8];
+      lo[c].get(a);
+      hi[c].get(b);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) ssq += lo[c][j] * lo[c][j] + hi[c][j] * hi[c][j];
+      for (int j = 0; j < 8; ++j) ssq += a[j] * a[j] + b[j] * b[j];
     }
   }
   return ssq;
 }
 
-template <int D>
+template <typename Tin, int D>
 __device__ __forceinline__ void norm_rotate_store(__nv_bfloat16 *row, const float *gain, int n_heads, float rinv,
-                                                  const float (&lo)[kMaxChunks][8], const float (&hi)[kMaxChunks][8],
-                                                  const float *s_cos, const float *s_sin) {
+                                                  const Chunk<Tin> (&lo)[kMaxChunks],
+                                                  const Chunk<Tin> (&hi)[kMaxChunks], const float *s_cos,
+                                                  const float *s_sin) {
   constexpr int CPH = D / 16;
 #pragma unroll
   for (int c = 0; c < kMaxChunks; ++c) {
     const int ci = threadIdx.x + c * kNormThreads;
     if (ci < n_heads * CPH) {
       const int h = ci / CPH, i0 = (ci % CPH) * 8;
-      float glo[8], ghi[8], ylo[8], yhi[8];
+      float glo[8], ghi[8], xlo[8], xhi[8], ylo[8], yhi[8];
       load8(gain + h * D + i0, glo);
       load8(gain + h * D + D / 2 + i0, ghi);
+      lo[c].get(xlo);
+      hi[c].get(xhi);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const float a = lo[c][j] * rinv * glo[j];
-        const float bb = hi[c][j] * rinv * ghi[j];
+        const float a = xlo[j] * rinv * glo[j];
+        const float bb = xhi[j] * rinv * ghi[j];
         const float cs = s_cos[i0 + j], sn = s_sin[i0 + j];
         ylo[j] = a * cs - bb * sn;
         yhi[j] = bb * cs + a * sn;
@@ -116,24 +150,26 @@ __global__ void __launch_bounds__(kNormThreads) qknorm_rope_kernel(
   const int b = static_cast<int>(tok / T);
   const int t = static_cast<int>(tok - static_cast<int64_t>(b) * T);
 
-  float qlo[kMaxChunks][8], qhi[kMaxChunks][8], klo[kMaxChunks][8], khi[kMaxChunks][8];
+  Chunk<Tin> qlo[kMaxChunks], qhi[kMaxChunks], klo[kMaxChunks], khi[kMaxChunks];
   const float ssq_q = load_row<Tin, D>(q + tok * H * D, H, qlo, qhi);
   const float ssq_k = load_row<Tin, D>(k + tok * G * D, G, klo, khi);
 
   if (threadIdx.x < D / 2) {
+    constexpr double kTwoPi = 6.283185307179586476925286766559;
     const double p = static_cast<double>(pos_offset[b]) + static_cast<double>(t);
-    double sn, cs;
-    sincos(p * tab.inv_freq[threadIdx.x], &sn, &cs);
-    s_cos[threadIdx.x] = static_cast<float>(cs) * tab.out_scale;
-    s_sin[threadIdx.x] = static_cast<float>(sn) * tab.out_scale;
+    const double a = p * tab.inv_freq[threadIdx.x];
+    float sn, cs;
+    sincosf(static_cast<float>(fma(-rint(a * (1.0 / kTwoPi)), kTwoPi, a)), &sn, &cs);
+    s_cos[threadIdx.x] = cs * tab.out_scale;
+    s_sin[threadIdx.x] = sn * tab.out_scale;
   }
   const float tq = block_sum(ssq_q, s_red[0]);
   const float tk = block_sum(ssq_k, s_red[1]);  // its __syncthreads also publishes s_cos / s_sin
   const float rq = 1.0f / sqrtf(tq / static_cast<float>(H * D) + eps);
   const float rk = 1.0f / sqrtf(tk / static_cast<float>(G * D) + eps);
 
-  norm_rotate_store<D>(q_out + tok * H * D, gain_q, H, rq, qlo, qhi, s_cos, s_sin);
-  norm_rotate_store<D>(k_out + tok * G * D, gain_k, G, rk, klo, khi, s_cos, s_sin);
+  norm_rotate_store<Tin, D>(q_out + tok * H * D, gain_q, H, rq, qlo, qhi, s_cos, s_sin);
+  norm_rotate_store<Tin, D>(k_out + tok * G * D, gain_k, G, rk, klo, khi, s_cos, s_sin);
 
   if (v_out != nullptr) {
     const Tin *vr = v + tok * G * D;
