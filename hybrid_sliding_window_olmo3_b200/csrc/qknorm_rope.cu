@@ -7,13 +7,14 @@
 // "Inference Pipeline" (RoPE at position offset + t) and "Technical Details"
 // (eps 1e-6; RoPE on queries and keys only).
 //
-// Memory-bound: every byte of q and k is read once and written once.  Each
-// thread owns "pair chunks" (8 features i..i+7 of a head and their rotation
-// partners i+d/2..i+d/2+7), loads them with 16-byte vector loads and keeps them in
-// registers across the block reduction of the sum of squares (bf16 inputs stay
-// packed, 4 registers per chunk, so that enough CTAs fit on an SM to keep HBM
-// busy).  64 threads form cos/sin once per token: the angle is reduced to
-// [-pi, pi] in fp64, then evaluated in fp32.
+// Memory-bound: q and k are read from HBM once and written once.  Each thread
+// owns "pair chunks" (8 features i..i+7 of a head and their rotation partners
+// i+d/2..i+d/2+7) and makes two passes over them with 16-byte vector loads: the
+// first sums their squares for the block-wide RMS, the second re-reads them (from
+// L2) to normalise, rotate and store.  Holding nothing across the reduction keeps
+// the kernel at 40 registers, 6 CTAs (tokens) per SM in flight.  64 threads form
+// cos/sin once per token: the angle is reduced to [-pi, pi] in fp64, then
+// evaluated in fp32.
 #include "common.cuh"
 #include "internal.h"
 
@@ -57,11 +58,21 @@ __device__ __forceinline__ float block_sum(float v, float *red) {
   return s;
 }
 
+
+// 16-byte load that bypasses L1 and that the compiler may not merge with an
+// earlier load of the same address (the second pass re-reads from L2).
+__device__ __forceinline__ uint4 ld_cg_u4(const void *p) {
+  uint4 u;
+  asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w) : "l"(p));
+  return u;
+}
+
 // Register copy of one pair chunk: packed bf16 (uint4) or 8 floats.
 template <typename Tin> struct Chunk;
 template <> struct Chunk<__nv_bfloat16> {
   uint4 u;
   __device__ __forceinline__ void load(const __nv_bfloat16 *p) { u = *reinterpret_cast<const uint4 *>(p); }
+  __device__ __forceinline__ void reload(const __nv_bfloat16 *p) { u = ld_cg_u4(p); }
   __device__ __forceinline__ void get(float (&x)[8]) const {
     float2 f;
     f = bf2_to_f2(u.x); x[0] = f.x; x[1] = f.y;
@@ -72,6 +83,7 @@ template <> struct Chunk<__nv_bfloat16> {
 };
 template <> struct Chunk<float> {
   float4 a, b;
+  __device__ __forceinline__ void reload(const float *p) { load(p); }
   __device__ __forceinline__ void load(const float *p) {
     a = reinterpret_cast<const float4 *>(p)[0];
     b = reinterpret_cast<const float4 *>(p)[1];
@@ -82,23 +94,22 @@ template <> struct Chunk<float> {
   }
 };
 
-// Loads the pair chunks of one row (n_heads heads) owned by this thread and
-// returns their sum of squares.
+// Sum of squares of this thread's pair chunks of one row, keeping nothing.
 template <typename Tin, int D>
-__device__ __forceinline__ float load_row(const Tin *row, int n_heads, Chunk<Tin> (&lo)[kMaxChunks],
-                                          Chunk<Tin> (&hi)[kMaxChunks]) {
-  constexpr int CPH = D / 16;  // pair chunks per head
+__device__ __forceinline__ float row_sumsq(const Tin *row, int n_heads) {
+  constexpr int CPH = D / 16;
   float ssq = 0.f;
 #pragma unroll
   for (int c = 0; c < kMaxChunks; ++c) {
     const int ci = threadIdx.x + c * kNormThreads;
     if (ci < n_heads * CPH) {
       const int h = ci / CPH, i0 = (ci % CPH) * 8;
-      lo[c].load(row + h * D + i0);
-      hi[c].load(row + h * D + D / 2 + i0);
+      Chunk<Tin> lo, hi;
+      lo.load(row + h * D + i0);
+      hi.load(row + h * D + D / 2 + i0);
       float a[8], b[8];
-      lo[c].get(a);
-      hi[c].get(b);
+      lo.get(a);
+      hi.get(b);
 #pragma unroll
       for (int j = 0; j < 8; ++j) ssq += a[j] * a[j] + b[j] * b[j];
     }
@@ -106,22 +117,25 @@ __device__ __forceinline__ float load_row(const Tin *row, int n_heads, Chunk<Tin
   return ssq;
 }
 
+// Second pass: re-read each chunk (from L2), normalise, rotate and store it.
 template <typename Tin, int D>
-__device__ __forceinline__ void norm_rotate_store(__nv_bfloat16 *row, const float *gain, int n_heads, float rinv,
-                                                  const Chunk<Tin> (&lo)[kMaxChunks],
-                                                  const Chunk<Tin> (&hi)[kMaxChunks], const float *s_cos,
-                                                  const float *s_sin) {
+__device__ __forceinline__ void reload_norm_rotate_store(const Tin *in_row, __nv_bfloat16 *row, const float *gain,
+                                                         int n_heads, float rinv, const float *s_cos,
+                                                         const float *s_sin) {
   constexpr int CPH = D / 16;
 #pragma unroll
   for (int c = 0; c < kMaxChunks; ++c) {
     const int ci = threadIdx.x + c * kNormThreads;
     if (ci < n_heads * CPH) {
       const int h = ci / CPH, i0 = (ci % CPH) * 8;
+      Chunk<Tin> lo, hi;
+      lo.reload(in_row + h * D + i0);
+      hi.reload(in_row + h * D + D / 2 + i0);
       float glo[8], ghi[8], xlo[8], xhi[8], ylo[8], yhi[8];
       load8(gain + h * D + i0, glo);
       load8(gain + h * D + D / 2 + i0, ghi);
-      lo[c].get(xlo);
-      hi[c].get(xhi);
+      lo.get(xlo);
+      hi.get(xhi);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const float a = xlo[j] * rinv * glo[j];
@@ -136,10 +150,10 @@ __device__ __forceinline__ void norm_rotate_store(__nv_bfloat16 *row, const floa
   }
 }
 
-// q_out / k_out may alias q / k: each element is read and written by the same
-// thread, and every read happens before the block-wide reduction.
+// q_out / k_out may alias q / k: each element is read (in both passes) and then
+// written by the same thread, and no other thread touches it.
 template <typename Tin, int D>
-__global__ void __launch_bounds__(kNormThreads) qknorm_rope_kernel(
+__global__ void __launch_bounds__(kNormThreads, sizeof(Tin) == 2 ? 6 : 1) qknorm_rope_kernel(
     const Tin *q, const Tin *k, const Tin *__restrict__ v, const float *__restrict__ gain_q,
     const float *__restrict__ gain_k, __nv_bfloat16 *q_out, __nv_bfloat16 *k_out, __nv_bfloat16 *__restrict__ v_out,
     const int32_t *__restrict__ pos_offset, int T, int H, int G, float eps, RopeTable tab) {
@@ -150,9 +164,8 @@ __global__ void __launch_bounds__(kNormThreads) qknorm_rope_kernel(
   const int b = static_cast<int>(tok / T);
   const int t = static_cast<int>(tok - static_cast<int64_t>(b) * T);
 
-  Chunk<Tin> qlo[kMaxChunks], qhi[kMaxChunks], klo[kMaxChunks], khi[kMaxChunks];
-  const float ssq_q = load_row<Tin, D>(q + tok * H * D, H, qlo, qhi);
-  const float ssq_k = load_row<Tin, D>(k + tok * G * D, G, klo, khi);
+  const float ssq_q = row_sumsq<Tin, D>(q + tok * H * D, H);
+  const float ssq_k = row_sumsq<Tin, D>(k + tok * G * D, G);
 
   if (threadIdx.x < D / 2) {
     constexpr double kTwoPi = 6.283185307179586476925286766559;
@@ -168,8 +181,8 @@ __global__ void __launch_bounds__(kNormThreads) qknorm_rope_kernel(
   const float rq = 1.0f / sqrtf(tq / static_cast<float>(H * D) + eps);
   const float rk = 1.0f / sqrtf(tk / static_cast<float>(G * D) + eps);
 
-  norm_rotate_store<Tin, D>(q_out + tok * H * D, gain_q, H, rq, qlo, qhi, s_cos, s_sin);
-  norm_rotate_store<Tin, D>(k_out + tok * G * D, gain_k, G, rk, klo, khi, s_cos, s_sin);
+  reload_norm_rotate_store<Tin, D>(q + tok * H * D, q_out + tok * H * D, gain_q, H, rq, s_cos, s_sin);
+  reload_norm_rotate_store<Tin, D>(k + tok * G * D, k_out + tok * G * D, gain_k, G, rk, s_cos, s_sin);
 
   if (v_out != nullptr) {
     const Tin *vr = v + tok * G * D;
