@@ -35,6 +35,7 @@
 // Every wait is bounded: on a timeout the CTA records OLMO3_DEVERR_TIMEOUT,
 // drains its copies and MMAs in flight, frees its tensor memory and exits.
 #include <math.h>
+#include <string.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -105,7 +106,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                         const __grid_constant__ CUtensorMap tmV, __nv_bfloat16 *__restrict__ out,
                         float *__restrict__ lse_out, int Tq, int Tk, int H, int G, int layer_type, int window,
                         float scale_log2, int n_blocks, const int32_t *__restrict__ pos_offset,
-                        const int64_t *__restrict__ seq_base, int *err) {
+                        const int64_t *__restrict__ seq_base, int *err,
+                        const __grid_constant__ PrefillExtraMaps xm) {
   using LY = PfLayout<D>;
   constexpr int NDB = D / 64;  // 64-feature (128-byte) blocks per row
   constexpr uint32_t IDESC_S = idesc_bf16_f32(kBM, kBN, 0);
@@ -136,6 +138,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   //                   it: keys are cache rows seq_base[b] + j, positions 0 .. qp0+Tq-1.
   //   kPrefillWindow  a chunk at pos_offset[b] over a gathered window: rows b*Tk + j
   //                   hold positions max(0, qp0 - window + 1) .. qp0 + Tq - 1.
+  //   kPrefillRing    the same keys read in place: a key tile of positions [P, P + 128)
+  //                   (P a multiple of 128, window a multiple of 128) comes from ring
+  //                   rows seq_base[b] + P mod window when P + 128 <= qp0, from chunk
+  //                   rows b*Tq + P - qp0 when P >= qp0, else from the bridge tile.
   // MODE is a template parameter so that the fresh-sequence kernel carries none
   // of the offset arithmetic (it costs registers in the softmax loop).
   int qp0 = 0, kp0 = 0, klen = Tk;
@@ -147,6 +153,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   } else if (MODE == kPrefillWindow) {
     kp0 = max(0, qp0 - window + 1);
     klen = qp0 + Tq - kp0;
+  } else if (MODE == kPrefillRing) {
+    kp0 = (max(0, qp0 - window + 1) / kBN) * kBN;  // key tiles start on 128-position boundaries
+    klen = qp0 + Tq - kp0;
+    krow0 = seq_base[b];
   }
 
   // key-tile ranges: the union [kt_lo, kt_lo + n_kt) and, per query tile w, [lo_w, hi_w] inside it
@@ -204,6 +214,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
+      if (MODE == kPrefillRing) {
+        prefetch_tmap(&xm.k_new);
+        prefetch_tmap(&xm.v_new);
+        prefetch_tmap(&xm.k_br);
+        prefetch_tmap(&xm.v_br);
+      }
       mbar_arrive_expect_tx(&q_full, 2 * LY::kQBytes);
 #pragma unroll
       for (int w = 0; w < 2; ++w)
@@ -218,8 +234,20 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           ok = false;
           break;
         }
-        const int krow = static_cast<int>(krow0 + static_cast<int64_t>(kt_lo + (i >> 1)) * kBN);
+        int krow = static_cast<int>(krow0 + static_cast<int64_t>(kt_lo + (i >> 1)) * kBN);
         const CUtensorMap *tm = (i & 1) ? &tmV : &tmK;
+        if (MODE == kPrefillRing) {
+          const int ts = kp0 + (kt_lo + (i >> 1)) * kBN;  // absolute position of the tile's first key
+          if (ts + kBN <= qp0) {
+            krow = static_cast<int>(krow0 + ts % window);
+          } else if (ts >= qp0) {
+            tm = (i & 1) ? &xm.v_new : &xm.k_new;
+            krow = b * Tq + (ts - qp0);
+          } else {
+            tm = (i & 1) ? &xm.v_br : &xm.k_br;
+            krow = b * kBN;
+          }
+        }
         mbar_arrive_expect_tx(&ring_full[slot], LY::kKVBytes);
 #pragma unroll
         for (int db = 0; db < NDB; ++db)
@@ -455,7 +483,7 @@ template <int D, int MODE>
 static cudaError_t launch_pf(const CUtensorMap &tmQ, const CUtensorMap &tmK, const CUtensorMap &tmV, void *out,
                              float *lse_out, int B, int Tq, int Tk, int H, int G, int layer_type, int window,
                              float scale, const int32_t *pos_offset, const int64_t *seq_base, int *err,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, const PrefillExtraMaps &xm) {
   using LY = PfLayout<D>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -468,7 +496,7 @@ static cudaError_t launch_pf(const CUtensorMap &tmQ, const CUtensorMap &tmK, con
   dim3 grid(H, n_blocks, B);
   attn_prefill_kernel<D, MODE><<<grid, kPfThreads, LY::kDynBytes, stream>>>(
       tmQ, tmK, tmV, static_cast<__nv_bfloat16 *>(out), lse_out, Tq, Tk, H, G, layer_type, window,
-      scale * 1.4426950408889634f, n_blocks, pos_offset, seq_base, err);
+      scale * 1.4426950408889634f, n_blocks, pos_offset, seq_base, err, xm);
   return cudaGetLastError();
 }
 
@@ -476,29 +504,38 @@ template <int D>
 static cudaError_t launch_pf_mode(int mode, const CUtensorMap &tmQ, const CUtensorMap &tmK, const CUtensorMap &tmV,
                                   void *out, float *lse_out, int B, int Tq, int Tk, int H, int G, int layer_type,
                                   int window, float scale, const int32_t *pos_offset, const int64_t *seq_base,
-                                  int *err, cudaStream_t stream) {
+                                  int *err, cudaStream_t stream, const PrefillExtraMaps &xm) {
   switch (mode) {
     case kPrefillFresh:
       return launch_pf<D, kPrefillFresh>(tmQ, tmK, tmV, out, lse_out, B, Tq, Tk, H, G, layer_type, window, scale,
-                                         pos_offset, seq_base, err, stream);
+                                         pos_offset, seq_base, err, stream, xm);
     case kPrefillCache:
       return launch_pf<D, kPrefillCache>(tmQ, tmK, tmV, out, lse_out, B, Tq, Tk, H, G, layer_type, window, scale,
-                                         pos_offset, seq_base, err, stream);
+                                         pos_offset, seq_base, err, stream, xm);
+    case kPrefillRing:
+      return launch_pf<D, kPrefillRing>(tmQ, tmK, tmV, out, lse_out, B, Tq, Tk, H, G, layer_type, window, scale,
+                                        pos_offset, seq_base, err, stream, xm);
     default:
       return launch_pf<D, kPrefillWindow>(tmQ, tmK, tmV, out, lse_out, B, Tq, Tk, H, G, layer_type, window, scale,
-                                          pos_offset, seq_base, err, stream);
+                                          pos_offset, seq_base, err, stream, xm);
   }
 }
 
 cudaError_t launch_attn_prefill(const CUtensorMap &tmQ, const CUtensorMap &tmK, const CUtensorMap &tmV, void *out,
                                 float *lse_out, int B, int Tq, int Tk, int H, int G, int d, int layer_type,
                                 int window, float scale, int mode, const int32_t *pos_offset,
-                                const int64_t *seq_base, int *err, cudaStream_t stream) {
+                                const int64_t *seq_base, int *err, cudaStream_t stream,
+                                const PrefillExtraMaps *extra) {
+  PrefillExtraMaps xm;
+  if (extra != nullptr)
+    xm = *extra;
+  else
+    memset(&xm, 0, sizeof(xm));
   if (d == 64)
     return launch_pf_mode<64>(mode, tmQ, tmK, tmV, out, lse_out, B, Tq, Tk, H, G, layer_type, window, scale,
-                              pos_offset, seq_base, err, stream);
+                              pos_offset, seq_base, err, stream, xm);
   return launch_pf_mode<128>(mode, tmQ, tmK, tmV, out, lse_out, B, Tq, Tk, H, G, layer_type, window, scale,
-                             pos_offset, seq_base, err, stream);
+                             pos_offset, seq_base, err, stream, xm);
 }
 
 }  // namespace olmo3

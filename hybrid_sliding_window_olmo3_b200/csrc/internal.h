@@ -50,12 +50,29 @@ constexpr int kPrefillBN = 128;  // keys per tile
 constexpr int kPrefillFresh = 0;   // the sequence itself, positions 0 .. T-1
 constexpr int kPrefillCache = 1;   // a linear cache already holding the chunk
 constexpr int kPrefillWindow = 2;  // a gathered window of a ring plus the chunk
+constexpr int kPrefillRing = 3;    // a ring read in place, the chunk, and one bridge tile
+
+// Extra key sources of kPrefillRing (3-d maps like tmK / tmV): the chunk's own
+// keys and values [B*T, G, d], and the bridge tile [B*128, G, d] that holds the
+// 128 positions around the chunk's start (ring rows before it, chunk rows after).
+struct PrefillExtraMaps {
+  CUtensorMap k_new, v_new, k_br, v_br;
+};
 
 // tmK / tmV are 3-d maps over [rows, G, d] with 64 x 1 x 128 boxes (128-byte swizzle).
+// For kPrefillRing, tmK / tmV map the cache [total_slots, G, d] and `extra` the other
+// sources; the window must be a multiple of kPrefillBN.  `extra` is ignored otherwise.
 cudaError_t launch_attn_prefill(const CUtensorMap &tmQ, const CUtensorMap &tmK, const CUtensorMap &tmV, void *out,
                                 float *lse_out, int B, int Tq, int Tk, int H, int G, int d, int layer_type,
                                 int window, float scale, int mode, const int32_t *pos_offset,
-                                const int64_t *seq_base, int *err, cudaStream_t stream);
+                                const int64_t *seq_base, int *err, cudaStream_t stream,
+                                const PrefillExtraMaps *extra = nullptr);
+
+// The bridge tile of kPrefillRing: rows j < 128 of [B, 128, G, d] hold position
+// 128 * floor(p0 / 128) + j: from the ring below p0, from the chunk from p0 on, zeros
+// past the chunk.
+cudaError_t launch_bridge_tile(const olmo3_kv_cache &c, const void *k_new, const void *v_new,
+                               const int32_t *pos_offset, int T, void *k_out, void *v_out, cudaStream_t stream);
 
 // Copies, for each sequence, the window of keys a chunk at pos_offset[b] needs:
 // rows j < Tk of [B, Tk, G, d] hold position max(0, p0 - window + 1) + j, from the

@@ -112,6 +112,48 @@ cudaError_t launch_gather_window(const olmo3_kv_cache &c, const void *k_new, con
   return cudaGetLastError();
 }
 
+// The one key tile of a sliding-layer chunk that straddles the chunk's start: the
+// 128 positions from 128 * floor(p0 / 128), taken from the ring below p0 and from
+// the chunk from p0 on (zeros past the chunk).  Every other key tile is read in
+// place, from the ring or from the chunk (attn_prefill.cu, kPrefillRing).
+__global__ void __launch_bounds__(kAppendThreads) bridge_tile_kernel(
+    const uint4 *__restrict__ ck, const uint4 *__restrict__ cv, const int64_t *__restrict__ seq_base,
+    int64_t total_slots, int window, int row_vec, const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new,
+    const int32_t *__restrict__ pos_offset, int T, uint4 *__restrict__ k_out, uint4 *__restrict__ v_out) {
+  const int j = blockIdx.x, b = blockIdx.y;
+  const int p0 = pos_offset[b];
+  const int p = (p0 >= 0 ? p0 / kPrefillBN : 0) * kPrefillBN + j;  // absolute position of this row
+  const uint4 *sk = nullptr, *sv = nullptr;
+  if (p < p0) {
+    const int64_t row = seq_base[b] + (p % window);
+    if (row >= 0 && row < total_slots) {
+      sk = ck + row * row_vec;
+      sv = cv + row * row_vec;
+    }
+  } else if (p0 >= 0 && p < p0 + T) {
+    const int64_t row = static_cast<int64_t>(b) * T + (p - p0);
+    sk = k_new + row * row_vec;
+    sv = v_new + row * row_vec;
+  }
+  uint4 *dk = k_out + (static_cast<int64_t>(b) * kPrefillBN + j) * row_vec;
+  uint4 *dv = v_out + (static_cast<int64_t>(b) * kPrefillBN + j) * row_vec;
+  const uint4 z = make_uint4(0, 0, 0, 0);
+  for (int i = threadIdx.x; i < row_vec; i += kAppendThreads) {
+    dk[i] = sk ? sk[i] : z;
+    dv[i] = sv ? sv[i] : z;
+  }
+}
+
+cudaError_t launch_bridge_tile(const olmo3_kv_cache &c, const void *k_new, const void *v_new,
+                               const int32_t *pos_offset, int T, void *k_out, void *v_out, cudaStream_t stream) {
+  const int row_vec = c.G * c.d * 2 / 16;
+  bridge_tile_kernel<<<dim3(kPrefillBN, c.B), kAppendThreads, 0, stream>>>(
+      static_cast<const uint4 *>(c.k), static_cast<const uint4 *>(c.v), c.seq_base, c.total_slots, c.window,
+      row_vec, static_cast<const uint4 *>(k_new), static_cast<const uint4 *>(v_new), pos_offset, T,
+      static_cast<uint4 *>(k_out), static_cast<uint4 *>(v_out));
+  return cudaGetLastError();
+}
+
 // "OLMo 3's Sliding-Window Attention Pattern", "The sliding-window mask": the
 // same predicate the attention kernels apply, written out as bytes.
 __global__ void attn_mask_kernel(int T, int window, int layer_type, uint8_t *__restrict__ out) {

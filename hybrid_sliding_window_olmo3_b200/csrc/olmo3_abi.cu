@@ -209,6 +209,8 @@ int olmo3_attn_prefill(const void *q, const void *k, const void *v, void *out, i
 size_t olmo3_attn_prefill_chunk_workspace_size(int B, int T, int G, int d, int layer_type, int window) {
   if (B < 0 || T < 0 || G < 1 || !valid_d(d) || !valid_type(layer_type) || window < 1) return 0;
   if (layer_type == OLMO3_FULL) return 0;
+  if (window % kPrefillBN == 0)  // the ring is read in place; only the bridge tile is copied
+    return 2 * static_cast<size_t>(B) * kPrefillBN * G * d * 2;
   return 2 * static_cast<size_t>(B) * (static_cast<size_t>(window) - 1 + T) * G * d * 2;
 }
 
@@ -243,7 +245,29 @@ int olmo3_attn_prefill_chunk(const void *q, const void *k_new, const void *v_new
     return cuda_status(launch_attn_prefill(tmQ, tmK, tmV, out, lse_out, B, T, 0, H, G, d, OLMO3_FULL, c->window,
                                            scale, kPrefillCache, pos_offset, c->seq_base, err_dev, s));
   }
-  // sliding: the ring's window and the chunk are gathered, attended, then the chunk is appended
+  if (c->window % kPrefillBN == 0) {
+    // sliding, window a multiple of the key tile: the chunk's rows read their keys in
+    // place, ring tiles from the cache and chunk tiles from k_new / v_new; only the
+    // tile that straddles the chunk's start is copied (the bridge); then the chunk is
+    // appended.
+    void *bk = workspace;
+    void *bv = static_cast<uint8_t *>(workspace) + need / 2;
+    PrefillExtraMaps xm;
+    if (!encode_kv(&tmK, c->k, c->total_slots, G, d) || !encode_kv(&tmV, c->v, c->total_slots, G, d) ||
+        !encode_kv(&xm.k_new, k_new, static_cast<int64_t>(B) * T, G, d) ||
+        !encode_kv(&xm.v_new, v_new, static_cast<int64_t>(B) * T, G, d) ||
+        !encode_kv(&xm.k_br, bk, static_cast<int64_t>(B) * kPrefillBN, G, d) ||
+        !encode_kv(&xm.v_br, bv, static_cast<int64_t>(B) * kPrefillBN, G, d))
+      return OLMO3_ERR_CUDA;
+    cudaError_t e = launch_bridge_tile(*c, k_new, v_new, pos_offset, T, bk, bv, s);
+    if (e != cudaSuccess) return OLMO3_ERR_CUDA;
+    e = launch_attn_prefill(tmQ, tmK, tmV, out, lse_out, B, T, 0, H, G, d, OLMO3_SLIDING, c->window, scale,
+                            kPrefillRing, pos_offset, c->seq_base, err_dev, s, &xm);
+    if (e != cudaSuccess) return OLMO3_ERR_CUDA;
+    return cuda_status(launch_kv_append(*c, k_new, v_new, pos_offset, T, nullptr, err_dev, s));
+  }
+  // sliding, any other window: the ring's window and the chunk are gathered side by
+  // side, attended, then the chunk is appended
   void *wk = workspace;
   void *wv = static_cast<uint8_t *>(workspace) + need / 2;
   if (!encode_kv(&tmK, wk, static_cast<int64_t>(B) * Tk, G, d) || !encode_kv(&tmV, wv, static_cast<int64_t>(B) * Tk, G, d))

@@ -206,10 +206,13 @@ int olmo3_attn_prefill(const void *q, const void *k, const void *v, void *out,
  *   Full layers: the chunk is appended first (it overwrites nothing), then the
  *   chunk attends over cache rows 0 .. pos_offset + T - 1; no workspace is used.
  *   Sliding layers: appending first would overwrite keys the chunk's early rows
- *   still need, so the window [pos_offset - window + 1, pos_offset) is gathered from
- *   the ring together with the chunk into `workspace`
- *   (olmo3_attn_prefill_chunk_workspace_size bytes), attended, then the chunk is
- *   appended.
+ *   still need, so the chunk attends first and is appended after.  When window is
+ *   a multiple of 128 the keys are read in place, 128-position tiles from the ring
+ *   before pos_offset and from k_new / v_new after it, and only the one tile that
+ *   straddles pos_offset is copied into `workspace`; for any other window the
+ *   window [pos_offset - window + 1, pos_offset) is gathered from the ring together
+ *   with the chunk into `workspace`.  Size: olmo3_attn_prefill_chunk_workspace_size
+ *   (2 * B * 128 * G * d * 2 bytes, or 2 * B * (window - 1 + T) * G * d * 2).
  *   Cache slots never written must hold finite values (allocate caches zeroed).
  *   err_dev as for olmo3_kv_append and olmo3_attn_prefill.
  */

@@ -150,7 +150,8 @@ def test_decode_workspace_and_validation(lib):
 def test_prefill_chunk_workspace_and_validation(lib):
     ws = L.attn_prefill_chunk_workspace_size
     assert ws(2, 100, 8, 128, L.FULL, 4096) == 0                      # full layers read the cache in place
-    assert ws(2, 100, 8, 128, L.SLIDING, 4096) == 2 * 2 * (4095 + 100) * 8 * 128 * 2
+    assert ws(2, 100, 8, 128, L.SLIDING, 4096) == 2 * 2 * 128 * 8 * 128 * 2       # ring read in place + bridge tile
+    assert ws(2, 100, 8, 128, L.SLIDING, 4000) == 2 * 2 * (3999 + 100) * 8 * 128 * 2  # other windows: gathered
     assert ws(2, 100, 8, 96, L.SLIDING, 4096) == 0                    # unsupported d
     f = lib.olmo3_attn_prefill_chunk
     f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(L.CacheStruct), ctypes.c_void_p,
