@@ -23,7 +23,7 @@ Sources (page title, section):
 * [SERVING]  "Olmo 3 7B" (inference-research record): per-layer-type cache
   management, KV bytes per token and "KV OVERPAY FOR THIS CHECKPOINT".
 
-Readings where the pages leave a step open (the same list is in the design doc):
+Readings where the pages leave a step open:
 
 * R1  RMSNorm puts eps inside the square root: x / sqrt(mean(x^2) + eps).
 * R2  QK-norm normalises the whole H*d query vector (G*d key vector) of a token.
@@ -37,6 +37,16 @@ Readings where the pages leave a step open (the same list is in the design doc):
 * R6  The cache stores keys after QK-norm and RoPE, at their absolute position.
 * R7  Ring slot = p mod window (sliding layers); linear slot = p (full layers).
 * R8  GQA: query head h reads key/value head floor(h / (H / G)).
+* R13 A prompt chunk at an offset attends over its cache and itself; on a sliding
+      layer it attends first and is appended after (appending first would
+      overwrite keys its early rows need).
+* R14 YaRN on full layers: NTK-by-parts frequencies with the method's ramp bounds
+      (beta_fast 32, beta_slow 1) and the temperature 0.1 ln(factor) + 1 on q and
+      k.  Parity unpinned beyond factor 1 (factor 1 is plain RoPE, pinned).
+* R15 Reordered norm: h = x + RMSNorm(attn W_o^T) over the D model features, one
+      gain per feature, eps 1e-6.
+* R16 The QKV projection takes the block input as it is (the reordered norm
+      leaves it un-normed).
 """
 from __future__ import annotations
 
