@@ -388,6 +388,7 @@ def _cache_from_oracle(ocs, typ, B, G, d, W, cap):
     (L.SLIDING, 256, 4, 2, 128, [256, 257, 600], 300),
     (L.SLIDING, 128, 10, 2, 128, [130, 5], 1),
     (L.SLIDING, 64, 2, 1, 64, [63, 64, 65], 77),
+    (L.SLIDING, 128, 4, 1, 64, [130, 0, 300], 77),   # d = 64 through the ring read in place
     (L.FULL, 4096, 4, 4, 128, [0, 5, 700], 129),
     (L.FULL, 4096, 10, 2, 128, [1000, 1], 300),
     (L.FULL, 4096, 2, 1, 64, [64, 3], 1),
