@@ -140,6 +140,53 @@ def check_attention_bruteforce(rng=np.random.default_rng(11)):
     return bool(ok)
 
 
+def check_reordered_norm(rng=np.random.default_rng(21)):
+    """[CASE] ingredient 6 fixes h = x + RMSNorm(attn W_o^T): the page's example (identity
+    W_o), and two consequences of the norm acting on the projected output before the
+    residual: h is unchanged when W_o is scaled, and h - x has RMS 1 (unit gains)."""
+    g = {r[0]: [float(x) for x in r[1:]] for r in read_golden("reordered_norm_example.txt")}
+    attn, x0 = np.array([g["attention_output"]]), np.array([[0.25, -2.0]])
+    ok = np.allclose(O.out_proj_postnorm_residual(x0, attn, np.eye(2), np.ones(2)) - x0, [g["added"]], atol=0.005)
+    x, a, w = rng.standard_normal((3, 8)), rng.standard_normal((3, 8)), rng.standard_normal((8, 8))
+    h1 = O.out_proj_postnorm_residual(x, a, w, np.ones(8), eps=0.0)  # eps 0: the invariances are exact
+    ok &= np.allclose(O.out_proj_postnorm_residual(x, a, 7.0 * w, np.ones(8), eps=0.0), h1, atol=1e-12)
+    ok &= np.allclose(np.sqrt(np.mean((h1 - x) ** 2, axis=-1)), 1.0, atol=1e-12)
+    return bool(ok)
+
+
+def check_qkv_identity(rng=np.random.default_rng(22)):
+    """Identity weights reduce the QKV projection to QK-norm + RoPE of the input's q and k
+    slices and hand the v slice through."""
+    B, T, H, G, d = 1, 3, 2, 1, 8
+    D = (H + 2 * G) * d
+    x = rng.standard_normal((B, T, D))
+    gq, gk = rng.uniform(0.5, 1.5, H * d), rng.uniform(0.5, 1.5, G * d)
+    pos = np.array([[4, 5, 6]])
+    qh, kh, v = O.qkv_projection(x, np.eye(D), gq, gk, pos, H, G, d)
+    rq, rk = O.qk_norm_rope(x[..., :H * d].reshape(B, T, H, d), x[..., H * d:(H + G) * d].reshape(B, T, G, d),
+                            gq, gk, pos)
+    return bool(np.allclose(qh, rq, atol=1e-12) and np.allclose(kh, rk, atol=1e-12) and
+                np.array_equal(v, x[..., (H + G) * d:].reshape(B, T, G, d)))
+
+
+def check_chunked_equals_one_shot(rng=np.random.default_rng(23)):
+    """A prompt fed in chunks through the cache gives the rows of the one-shot prefill
+    ([README] "Inference Pipeline"), for a ring shorter than the prompt too."""
+    ok = True
+    B, H, G, d, Ttot = 1, 2, 1, 4, 11
+    q, k, v = (rng.standard_normal((B, Ttot, n, d)) for n in (H, G, G))
+    for typ, W in (("sliding", 3), ("full", 3)):
+        ref, _ = O.prefill_attention(q, k, v, typ, W)
+        cache = O.KVCache(typ, W if typ == "sliding" else Ttot, G, d)
+        p0 = 0
+        for T in (4, 1, 6):
+            o, _ = O.chunk_attention(q[:, p0:p0 + T], k[:, p0:p0 + T], v[:, p0:p0 + T], [cache], [p0], typ, W)
+            ok &= np.allclose(o, ref[:, p0:p0 + T], atol=1e-12)
+            cache.append(range(p0, p0 + T), k[0, p0:p0 + T], v[0, p0:p0 + T])
+            p0 += T
+    return bool(ok)
+
+
 # ----------------------------------------------------------------------------
 # Pins
 # ----------------------------------------------------------------------------
@@ -497,9 +544,44 @@ def _mut_attend_no_scale(q, q_pos, k, k_pos, v, layer_type, window, scale=None, 
     return _real_attend(q, q_pos, k, k_pos, v, layer_type, window, 1.0, k_valid)
 
 
+def _mut_postnorm_before_projection(x, attn, w_o, gain, eps=1e-6):
+    # the norm on the attention output before W_o
+    return np.asarray(x, np.float64) + O.rms_norm(np.asarray(attn, np.float64), np.ones(np.shape(attn)[-1]),
+                                                   eps) @ np.asarray(w_o, np.float64).T * np.asarray(gain)
+
+
+def _mut_postnorm_residual_inside(x, attn, w_o, gain, eps=1e-6):
+    # the residual added before the norm (pre-norm-like order)
+    y = np.asarray(x, np.float64) + np.asarray(attn, np.float64) @ np.asarray(w_o, np.float64).T
+    return O.rms_norm(y, gain, eps)
+
+
+_real_qkv = O.qkv_projection
+
+
+def _mut_qkv_k_v_swapped(x, w_qkv, gain_q, gain_k, positions, H, G, d, *args, **kw):
+    w = np.asarray(w_qkv, np.float64)
+    w = np.concatenate([w[:H * d], w[(H + G) * d:], w[H * d:(H + G) * d]])
+    return _real_qkv(x, w, gain_q, gain_k, positions, H, G, d, *args, **kw)
+
+
+def _mut_qkv_prenormed_input(x, w_qkv, gain_q, gain_k, positions, H, G, d, *args, **kw):
+    x = np.asarray(x, np.float64)
+    return _real_qkv(O.rms_norm(x, np.ones(x.shape[-1])), w_qkv, gain_q, gain_k, positions, H, G, d, *args, **kw)
+
+
+_real_chunk = O.chunk_attention
+
+
+def _mut_chunk_ignores_cache(q_hat, k_hat, v, caches, pos_offset, layer_type, window, scale=None):
+    empty = [O.KVCache(c.layer_type, c.n_slots, c.k.shape[1], c.k.shape[2]) for c in caches]
+    return _real_chunk(q_hat, k_hat, v, empty, pos_offset, layer_type, window, scale)
+
+
 ALL_CHECKS = [check_mask_table, check_layer_type_examples, check_window3_token4,
               check_qknorm_example, check_rope_slowest_pair, check_rope_pairing,
-              check_gqa_equals_repeated_mha, check_attention_bruteforce]
+              check_gqa_equals_repeated_mha, check_attention_bruteforce,
+              check_reordered_norm, check_qkv_identity, check_chunked_equals_one_shot]
 
 
 def test_all_checks_pass_on_the_oracle():
@@ -514,6 +596,11 @@ def test_all_checks_pass_on_the_oracle():
     ("rope", _mut_rope_adjacent),
     ("attend", _mut_attend_gqa_modulo),
     ("attend", _mut_attend_no_scale),
+    ("out_proj_postnorm_residual", _mut_postnorm_before_projection),
+    ("out_proj_postnorm_residual", _mut_postnorm_residual_inside),
+    ("qkv_projection", _mut_qkv_k_v_swapped),
+    ("qkv_projection", _mut_qkv_prenormed_input),
+    ("chunk_attention", _mut_chunk_ignores_cache),
 ])
 def test_planted_mistakes_are_caught(monkeypatch, name, mut):
     monkeypatch.setattr(O, name, mut)
