@@ -13,7 +13,14 @@ as the max over ranks.  With several GPUs every rank runs an independent
 replica (the path has no data-path exchange): scaling is weak.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload 7b-prefill|32b-prefill|7b-decode|32b-decode|ragged-7b-decode]
+                  [--workload 7b-prefill|32b-prefill|7b-decode|32b-decode|ragged-7b-decode|
+                              7b-prefill-chunked|32b-prefill-chunked|7b-qkv-proj|32b-qkv-proj|
+                              7b-out-proj|32b-out-proj]
+
+The chunked workloads feed the prefill prompt through the chunked-prefill call
+(--chunk tokens at a time); the projection workloads time the attention block's
+fused QKV projection (+ QK-norm + RoPE) and output side (W_o + reordered norm +
+residual) over the prefill workloads' tokens.
 """
 from __future__ import annotations
 
