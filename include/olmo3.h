@@ -2,13 +2,15 @@
  * olmo3.h - C ABI of the OLMo 3 hybrid sliding-window attention library (libolmo3.so).
  *
  * The library computes, on one B200 (sm_100a), the attention hot path of OLMo 3
- * inference as the pages define it:
+ * inference as the pages define it, and the attention block's two projections with
+ * their norms fused in:
  *
  *   [PATTERN] "OLMo 3's Sliding-Window Attention Pattern" (scratchllm.com problem page):
  *             "Which layers are full", "The sliding-window mask", "Hint".
  *   [CASE]    "Case Study: OLMo 3" (scratchllm.com learn page), "The architecture":
- *             ingredient 1 (GQA), 2 (QK-norm), 3 (RoPE, theta = 500,000, rotate half),
- *             4 (sliding-window attention).
+ *             ingredient 1 (bias-free projections, GQA), 2 (QK-norm), 3 (RoPE,
+ *             theta = 500,000, rotate half), 4 (sliding-window attention),
+ *             6 (reordered norm), 7 (YaRN on the full layers of the long-context model).
  *   [COUNT]   "Count OLMo 3's Parameters" (scratchllm.com), "What to count":
  *             QK-norm gains of sizes H*d and G*d.
  *   [README]  "Olmo-3 End-to-End Implementation" (GitHub README): "Inference Pipeline",
